@@ -1,0 +1,421 @@
+"""GQLA decode-attention benchmark (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--sq 1|2] [--impl ours|reference]
+
+Workload: the LLaMA-3-8B-shaped GQLA layer (n_h 32, G 8, d_nope 128, d_rope
+64, d_v 128, r 512), batch 32, uniform context 8192, s_q new tokens per
+sequence, bf16, synthetic seeded inputs.  One step is one pass of the whole
+decode hot path over that batch: the decode-time expansion of the s_q new
+tokens into the per-group cache, the MQA-absorb decode and the GQA decode
+(both paths produce the batch's B*s_q output tokens).  value = decoded tokens
+(B*s_q per step, per GPU) / device time.  Under torchrun every rank decodes
+its own batch (weak scaling; sequences are independent, no data-path
+collective); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this build)
+on the same workload, one bounded sample of (sequence, group) units per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode attention tokens/s per layer and % of roofline (HBM GB/s or TC util), 1×B200"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--sq", type=int, default=1, choices=[1, 2])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def workload(s_q):
+    from latent_kv_cache_flash_b200 import synth
+    return synth.llama3_8b(s_q=s_q)
+
+
+def algorithmic(wl):
+    """Per-step algorithmic bytes and flops of each path (the method's own
+    traffic: cache bytes read once per step, q/out/weights ignored)."""
+    d = wl.dims
+    T = wl.batch * wl.seq_len
+    keys = sum(wl.seq_len - d.s_q + i + 1 for i in range(d.s_q)) * wl.batch   # (query, key) pairs per head
+    absorb_bytes = 2 * T * (d.r + d.d_rope)
+    absorb_flops = d.n_h * keys * 2 * (2 * d.r + d.d_rope) + wl.batch * d.s_q * d.n_h * 2 * d.r * (d.d_nope + d.d_v)
+    gqa_bytes = 2 * T * d.G * (d.d_qk + d.d_v)
+    gqa_flops = d.n_h * keys * 2 * (d.d_qk + d.d_v)
+    return dict(absorb_bytes=absorb_bytes, absorb_flops=absorb_flops, gqa_bytes=gqa_bytes, gqa_flops=gqa_flops)
+
+
+# ---------------------------------------------------------------- clocks ---
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.idx = gpu_index
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench.csv") if os.path.isdir(
+            os.path.join(ROOT, "gpurun_out")) else "/tmp/gqla_clocks.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-i", str(self.idx), "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx = float(p[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------- cpu baseline ---
+def oracle_sample(inp, units, both_forms=True):
+    """Runs the oracle on (sequence, group) units; returns seconds."""
+    import numpy as np
+    from oracle import gqla_oracle as O
+    d = inp.dims
+    W_uk = inp.W_uk.double().cpu().numpy()
+    W_uv = inp.W_uv.double().cpu().numpy()
+    t0 = time.perf_counter()
+    for b, g in units:
+        rows = inp.logical_latent(b).double().cpu().numpy()
+        qb = inp.q[b].double().cpu().numpy()
+        L = inp.seq_lens_host[b]
+        O.decode_sequence_gqa(qb, rows[:, :d.r], rows[:, d.r:], W_uk, W_uv, L, d.softmax_scale, groups=[g])
+        if both_forms:
+            O.decode_sequence_absorb(qb, rows[:, :d.r], rows[:, d.r:], W_uk, W_uv, L, d.softmax_scale, groups=[g])
+    return time.perf_counter() - t0
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(inp, budget_s=12.0):
+    wl = inp.wl
+    d = wl.dims
+    all_units = [(b, g) for b in range(wl.batch) for g in range(d.G)]
+    import random
+    rnd = random.Random(0)
+    rnd.shuffle(all_units)
+    done, spent = 0, 0.0
+    while done < len(all_units) and (spent < budget_s or done < 2):
+        spent += oracle_sample(inp, [all_units[done]])
+        done += 1
+    per_step = spent / done * len(all_units)
+    return {"value": wl.batch * d.s_q / per_step, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": "%d of %d (sequence, group) units of %s (B%d L%d s_q%d), fp64 expanded and absorb forms, "
+                      "%.1f s, extrapolated linearly to the whole batch" % (
+                          done, len(all_units), wl.name, wl.batch, wl.seq_len, d.s_q, spent)}
+
+
+# ----------------------------------------------------------- reference ---
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from latent_kv_cache_flash_b200 import synth
+    wl = workload(args.sq)
+    inp = synth.make_inputs(wl, "cpu")
+    d = wl.dims
+    all_units = [(b, g) for b in range(wl.batch) for g in range(d.G)]
+    # one unit per step keeps the whole run within a few minutes
+    for w in range(args.warmup):
+        oracle_sample(inp, [all_units[w % len(all_units)]])
+    t = 0.0
+    for s in range(args.steps):
+        t += oracle_sample(inp, [all_units[(args.warmup + s) % len(all_units)]])
+    per_unit = t / args.steps
+    step_s = per_unit * len(all_units)
+    value = wl.batch * d.s_q / step_s
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "%s B%d L%d s_q%d" % (wl.name, wl.batch, wl.seq_len, d.s_q), "batch": wl.batch,
+                       "seq_len": wl.seq_len, "s_q": d.s_q, "n_h": d.n_h, "G": d.G, "r": d.r},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": "one (sequence, group) unit per step, fp64 expanded and absorb forms, "
+                                       "extrapolated to %d units per step" % len(all_units)},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ ours ---
+def kernel_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "latent_kv_cache_flash_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_name):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        rec = json.load(open(p)).get(kernel_name)
+    except Exception:
+        return None
+    if not rec or rec.get("source_sha") != kernel_sha():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from latent_kv_cache_flash_b200 import build, gqla, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    build.build()
+    hbm, tf_burst, tf_sust, peak_src = load_peaks()
+
+    wl = workload(args.sq)
+    wl.seed = wl.seed + rank
+    d = wl.dims
+    inp = synth.make_inputs(wl, dev)
+    dims = gqla.make_dims(d)
+    lay = gqla.make_layout(inp.seq_lens, inp.max_seq_len, 0, inp.capacity, None, 0)
+    ks, vs = synth.expanded_pool_shapes(inp)
+    kp = torch.empty(ks, dtype=d.torch_dtype, device=dev)
+    vp = torch.empty(vs, dtype=d.torch_dtype, device=dev)
+    B = wl.batch
+    out_a = torch.empty((B, d.s_q, d.n_h, d.d_v), dtype=d.torch_dtype, device=dev)
+    out_g = torch.empty_like(out_a)
+    lse_a = torch.empty((B, d.s_q, d.n_h), device=dev)
+    lse_g = torch.empty_like(lse_a)
+    ws_a = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_ABSORB, dev)
+    ws_g = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_GQA, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # the resident per-group cache of all tokens (a prefill-time cost, timed on its own)
+    gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0, status)
+
+    def expand_tail():
+        gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, d.s_q, status)
+
+    def absorb():
+        gqla.gqla_decode_absorb(dims, lay, inp.q, inp.latent, inp.W_uk, inp.W_uv, out_a, lse_a, 0, ws_a, status)
+
+    def gqa():
+        gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out_g, lse_g, 0, ws_g, status)
+
+    def step():
+        expand_tail()
+        absorb()
+        gqa()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(fn, n):
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    n0 = gqla.gqla_launch_counter()
+    total_ms = timed(step, args.steps)
+    launches = gqla.gqla_launch_counter() - n0
+    ms_step = total_ms / args.steps
+    # per-call breakdown (each over at least ~0.3 s of device time)
+    reps = max(args.steps, int(300.0 / max(ms_step, 1e-3)))
+    ms_absorb = timed(absorb, reps) / reps
+    ms_gqa = timed(gqa, reps) / reps
+    ms_tail = timed(expand_tail, reps) / reps
+    ms_expand_full = timed(lambda: gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0,
+                                                          status), 3) / 3
+
+    # end to end through the public API with host buffers: the step's new
+    # inputs (queries and the new tokens' latent rows) go host->device, both
+    # paths' outputs come back device->host, inside the timed region
+    q_host = inp.q.cpu().pin_memory()
+    Lmax = wl.seq_len
+    new_rows_host = inp.latent[:, Lmax - d.s_q:Lmax].cpu().pin_memory()
+    out_host = torch.empty((2,) + tuple(out_a.shape), dtype=out_a.dtype).pin_memory()
+
+    def e2e_step():
+        inp.q.copy_(q_host, non_blocking=True)
+        inp.latent[:, Lmax - d.s_q:Lmax].copy_(new_rows_host, non_blocking=True)
+        step()
+        out_host[0].copy_(out_a, non_blocking=True)
+        out_host[1].copy_(out_g, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    e2e_ms = timed(e2e_step, args.steps) / args.steps
+    clk = clocks.stop() if clocks else None
+    torch.cuda.synchronize()
+    st = int(status.item())
+    if st != 0:
+        raise SystemExit("device status 0x%x during the bench" % st)
+
+    alg = algorithmic(wl)
+    tokens = B * d.s_q
+    value = world * tokens / (ms_step * 1e-3)
+    # dominant kernel: the slower decode call of the step
+    if ms_gqa >= ms_absorb:
+        name, ms_dom, bytes_dom = "gqla_decode_gqa", ms_gqa, alg["gqa_bytes"]
+        roof = {"bound": "hbm", "achieved": bytes_dom / (ms_dom * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s"}
+    else:
+        name, ms_dom = "gqla_decode_absorb", ms_absorb
+        t_hbm = alg["absorb_bytes"] / (hbm * 1e9)
+        t_tc = alg["absorb_flops"] / (tf_burst * 1e12)
+        if t_hbm >= t_tc:
+            roof = {"bound": "hbm", "achieved": alg["absorb_bytes"] / (ms_dom * 1e-3) / 1e9, "peak": hbm,
+                    "unit": "GB/s"}
+        else:
+            roof = {"bound": "tensor", "achieved": alg["absorb_flops"] / (ms_dom * 1e-3) / 1e12, "peak": tf_burst,
+                    "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic(name)
+    roof["kernel"] = name
+    roof["peak_source"] = peak_src
+
+    def path_entry(ms, nbytes, flops):
+        t_roof = max(nbytes / (hbm * 1e9), flops / (tf_burst * 1e12))
+        return {"ms": ms, "tokens_per_s": tokens / (ms * 1e-3), "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+                "tflops": flops / (ms * 1e-3) / 1e12, "roofline_frac": t_roof / (ms * 1e-3),
+                "bound": "hbm" if nbytes / (hbm * 1e9) >= flops / (tf_burst * 1e12) else "tensor"}
+
+    T = B * wl.seq_len
+    exp_flops = 2 * T * d.r * d.G * (d.d_nope + d.d_v)
+    exp_bytes = 2 * T * (d.r + d.d_rope) + 2 * T * d.G * (d.d_qk + d.d_v)
+    h2d = q_host.numel() * q_host.element_size() + new_rows_host.numel() * new_rows_host.element_size()
+    d2h = out_host.numel() * out_host.element_size()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, random-init weights)",
+        "config": {"workload": "%s B%d L%d s_q%d" % (wl.name, B, wl.seq_len, d.s_q), "batch": B,
+                   "seq_len": wl.seq_len, "s_q": d.s_q, "n_h": d.n_h, "G": d.G, "d_nope": d.d_nope,
+                   "d_rope": d.d_rope, "d_v": d.d_v, "r": d.r,
+                   "step": "expand s_q new tokens + absorb decode + GQA decode",
+                   "l2": "no flush: inputs larger than L2 (latent %.0f MB, expanded cache %.0f MB)" % (
+                       alg["absorb_bytes"] / 1e6, alg["gqa_bytes"] / 1e6),
+                   "parallelism": "replicas x%d (batch-sharded, no collective)" % world},
+        "roofline": roof,
+        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "paths": {"absorb": path_entry(ms_absorb, alg["absorb_bytes"], alg["absorb_flops"]),
+                  "gqa": path_entry(ms_gqa, alg["gqa_bytes"], alg["gqa_flops"]),
+                  "expand_tail": {"ms": ms_tail},
+                  "expand_full_cache": {"ms": ms_expand_full, "tflops": exp_flops / (ms_expand_full * 1e-3) / 1e12,
+                                        "hbm_gbs": exp_bytes / (ms_expand_full * 1e-3) / 1e9,
+                                        "tc_frac": exp_flops / (ms_expand_full * 1e-3) / (tf_burst * 1e12)}},
+        "splits": {"absorb": gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_ABSORB),
+                   "gqa": gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_GQA)},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = inp
+        line["cpu_baseline"] = cpu_baseline(inp_cpu)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,205 @@
+/*
+ * gqla.h -- C ABI of the GQLA decode-attention library (libgqla.so, sm_100a).
+ *
+ * Group-Query Latent Attention keeps one joint latent c_KV (rank r) and one
+ * decoupled RoPE key k_rope per cached token, and group-shared up-projections
+ * W_uk^g, W_uv^g (one pair per group of m = n_h / G query heads).  The same
+ * weights decode two ways ("GQLA: Group-Query Latent Attention for
+ * Hardware-Adaptive Decoding", scholarbro.com, Abstract; "GQLA" on
+ * chatpaper.ai, Abstract): the MQA-absorb path attends every head over the
+ * latent cache with the query carried through W_uk^g, and the GQA path expands
+ * the latent into a per-group K/V cache and runs grouped-query decode over it.
+ * Both give, for batch b, new token i in [0, s_q) and head h in group g:
+ *
+ *     k_{g,t} = [ c_t W_uk^g ; k_rope_t ]      v_{g,t} = c_t W_uv^g
+ *     s_t = scale * <q_{b,i,h}, k_{g,t}>        for t = 0 .. L_b - s_q + i
+ *     out_{b,i,h} = sum_t softmax(s)_t v_{g,t}  lse_{b,i,h} = ln sum_t exp(s_t)
+ *
+ * Conventions shared by every entry point:
+ *  - All pointers named *device* are CUDA device pointers owned by the caller;
+ *    the library never allocates device memory (split-KV scratch is passed in
+ *    as a workspace) and never frees anything.  Host structs are read during
+ *    the call only.
+ *  - Work is queued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *    and runs asynchronously; no call synchronises.
+ *  - Arguments are validated on the host before any launch; a failed check
+ *    returns a status and launches nothing.  A kernel launch failure returns
+ *    GQLA_ERR_CUDA.
+ *  - Problems only the device can see (a sequence shorter than s_q or longer
+ *    than its slots, a page id outside the pool) set bits in *dev_status
+ *    (device int32, may be NULL) and the affected rows are written as zeros with
+ *    lse = -inf; the kernel never traps.
+ *  - Element type of q, caches, weights and out is dims.dtype (fp32 or bf16);
+ *    lse and all accumulation are fp32.  The fp32 kernels compute in true fp32
+ *    (no TF32); the bf16 kernels use tensor cores with fp32 accumulation.
+ *  - Row-major layouts:
+ *      q       [B, s_q, n_h, d_nope + d_rope]       nope part first
+ *      latent  token rows [c_KV (r) ; k_rope (d_rope)]
+ *      K pool  token rows [G, d_nope + d_rope]      (per-group key with its own
+ *                                                     copy of k_rope)
+ *      V pool  token rows [G, d_v]
+ *      W_uk    [G, r, d_nope]      W_uv [G, r, d_v]
+ *      out     [B, s_q, n_h, d_v]  lse [B, s_q, n_h]
+ *    Head h belongs to group h / m.  Rotary embedding is applied before these
+ *    calls (q_rope and k_rope arrive rotated).
+ */
+#ifndef GQLA_H
+#define GQLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gqla_status {
+  GQLA_OK = 0,
+  GQLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, n_h % G != 0, s_q out of [1,4] */
+  GQLA_ERR_UNSUPPORTED = 2,  /* valid GQLA dims no kernel of this build handles */
+  GQLA_ERR_ALIGNMENT = 3,    /* a pointer or row pitch below the 16-byte rule */
+  GQLA_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than gqla_workspace_bytes */
+  GQLA_ERR_CUDA = 5          /* a CUDA call or kernel launch failed */
+} gqla_status;
+
+typedef enum gqla_dtype { GQLA_F32 = 0, GQLA_BF16 = 1 } gqla_dtype;
+
+typedef enum gqla_path { GQLA_PATH_ABSORB = 0, GQLA_PATH_GQA = 1 } gqla_path;
+
+/* Device status bits written to *dev_status (OR-ed). */
+#define GQLA_DEV_SHORT_SEQ 1   /* seq_lens[b] < s_q (or < 0): rows of b zeroed  */
+#define GQLA_DEV_OVERFLOW 2    /* seq_lens[b] above the sequence's token slots  */
+#define GQLA_DEV_BAD_PAGE 4    /* block_table entry outside [0, num_pages)      */
+#define GQLA_DEV_TIMEOUT 8     /* a bounded pipeline wait gave up               */
+
+/* Model dimensions of one attention layer.  The group count must divide n_h
+ * ("gqla_attn" module page, frankenstein-transformer docs: GQLAAttention
+ * raises when gqla_num_groups does not divide num_heads).  scale multiplies
+ * <q, k> (commonly 1/sqrt(d_nope + d_rope)); s_q is the number of new tokens
+ * per sequence decoded in one step (multi-token prediction, 1..4). */
+typedef struct gqla_dims {
+  int32_t n_h;      /* query heads                                   */
+  int32_t G;        /* groups (KV heads of the expanded path)        */
+  int32_t d_nope;   /* per-head query/key dims without RoPE          */
+  int32_t d_rope;   /* shared decoupled-RoPE key dims                */
+  int32_t d_v;      /* value dims per head                           */
+  int32_t r;        /* latent rank of c_KV                           */
+  int32_t s_q;      /* new tokens per sequence, 1..4                 */
+  float scale;      /* softmax scale                                 */
+  gqla_dtype dtype; /* element type of q, caches, weights and out    */
+} gqla_dims;
+
+/* Where token t of sequence b lives in a token pool (the same geometry serves
+ * the latent pool and the expanded K and V pools).  A pool is an array of
+ * token rows; `row` below is that pool's row width in elements.
+ *   contiguous (page_size == 0): pool [batch, capacity, row]; token (b, t) is
+ *     row b * capacity + t.
+ *   paged (page_size > 0): pool [num_pages, page_size, row]; token (b, t) is
+ *     row block_table[b * max_blocks_per_seq + t / page_size] * page_size
+ *     + t % page_size (fixed-size blocks as in PagedAttention, "Grouped Query
+ *     Attention (GQA)" glossary, section "GQA et techniques connexes").
+ * seq_lens[b] counts all tokens of sequence b, its s_q new tokens included;
+ * slots past it may hold any finite values. */
+typedef struct gqla_kv_layout {
+  int32_t batch;                /* B > 0                                      */
+  const int32_t* seq_lens;      /* device [batch]                              */
+  int32_t max_seq_len;          /* host upper bound on seq_lens (plans splits) */
+  int32_t page_size;            /* 0 = contiguous; else tokens per page        */
+  int32_t capacity;             /* contiguous: token slots per sequence        */
+  const int32_t* block_table;   /* paged: device [batch, max_blocks_per_seq]   */
+  int32_t max_blocks_per_seq;   /* paged: columns of block_table               */
+  int32_t num_pages;            /* paged: pages in the pool                    */
+} gqla_kv_layout;
+
+/* Per-group cache expansion, the GQA path's precondition ("GQLA" chatpaper.ai
+ * Abstract: a GQA path with a per-group expanded cache):
+ *   K[b,t,g,:] = [ c_{b,t} W_uk^g ; k_rope_{b,t} ],  V[b,t,g,:] = c_{b,t} W_uv^g
+ * for tokens t in [max(0, seq_lens[b] - tail_tokens), seq_lens[b]) of every
+ * sequence (tail_tokens <= 0: all tokens).  tail_tokens = s_q expands just the
+ * tokens appended by one decode step.
+ *   latent  device, pool with rows of r + d_rope elements
+ *   W_uk    device [G, r, d_nope];  W_uv device [G, r, d_v]
+ *   k_pool  device, pool with rows of G*(d_nope+d_rope) elements (written)
+ *   v_pool  device, pool with rows of G*d_v elements (written)
+ * All three pools use `layout`.  Rows outside the expanded range are not
+ * touched. */
+gqla_status gqla_expand_cache(const gqla_dims* dims, const gqla_kv_layout* layout,
+                              const void* latent, const void* W_uk, const void* W_uv,
+                              void* k_pool, void* v_pool, int32_t tail_tokens,
+                              int32_t* dev_status, void* stream);
+
+/* MQA-absorb decode ("GQLA" chatpaper.ai Abstract: an MQA-absorb path
+ * identical to MLA's).  Per head: q~ = W_uk^g q_nope, scores
+ * scale*(<q~, c_t> + <q_rope, k_rope_t>), latent output sum_t p_t c_t, then
+ * out = that latent output times W_uv^g.
+ *   q        device [B, s_q, n_h, d_nope + d_rope]
+ *   latent   device pool, rows of r + d_rope
+ *   out      device [B, s_q, n_h, d_v] (written)
+ *   lse      device fp32 [B, s_q, n_h] or NULL
+ *   num_splits  key-range splits per sequence, 0 = chosen by the library
+ *   workspace   device, >= gqla_workspace_bytes(dims, layout, num_splits,
+ *               GQLA_PATH_ABSORB) bytes, 256-byte aligned; contents clobbered */
+gqla_status gqla_decode_absorb(const gqla_dims* dims, const gqla_kv_layout* layout,
+                               const void* q, const void* latent,
+                               const void* W_uk, const void* W_uv,
+                               void* out, float* lse, int32_t num_splits,
+                               void* workspace, size_t workspace_bytes,
+                               int32_t* dev_status, void* stream);
+
+/* GQA decode over the expanded per-group cache ("GQLA" chatpaper.ai Abstract;
+ * grouped-query attention as in the "Grouped Query Attention (GQA)" glossary,
+ * section "Fonctionnement de la GQA": every head of group g attends over the
+ * group's K/V).
+ *   q       device [B, s_q, n_h, d_nope + d_rope]
+ *   k_pool  device pool, rows of G*(d_nope+d_rope);  v_pool rows of G*d_v
+ *   out, lse, num_splits, workspace as for gqla_decode_absorb (path GQA). */
+gqla_status gqla_decode_gqa(const gqla_dims* dims, const gqla_kv_layout* layout,
+                            const void* q, const void* k_pool, const void* v_pool,
+                            void* out, float* lse, int32_t num_splits,
+                            void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream);
+
+/* Log-sum-exp merge of attention results over disjoint key ranges:
+ *   lse[row] = ln sum_j exp(lse_part[j,row]);
+ *   out[row] = sum_j exp(lse_part[j,row] - lse[row]) * o_part[j,row,:]
+ * A part with lse = -inf has weight 0; a row whose parts are all -inf gets
+ * out = 0, lse = -inf.  (The pages name FlashAttention-style kernels --
+ * "Grouped Query Attention (GQA)" glossary, "GQA et techniques connexes" --
+ * but print no merge rule; this is the identity softmax obeys.)
+ *   o_part   device fp32 [num_splits, rows, D];  lse_part device fp32 [num_splits, rows]
+ *   out      device [rows, D] of out_dtype;      lse_out device fp32 [rows] or NULL */
+gqla_status gqla_splitkv_combine(int32_t num_splits, int32_t rows, int32_t D,
+                                 const float* o_part, const float* lse_part,
+                                 void* out, gqla_dtype out_dtype, float* lse_out,
+                                 void* stream);
+
+/* Workspace bytes a decode call needs (0 when none), for the given split count
+ * (0 = the library's choice, the same one the decode call will make). */
+size_t gqla_workspace_bytes(const gqla_dims* dims, const gqla_kv_layout* layout,
+                            int32_t num_splits, gqla_path path);
+
+/* Split count a decode call with this num_splits argument will use. */
+int32_t gqla_num_splits(const gqla_dims* dims, const gqla_kv_layout* layout,
+                        int32_t num_splits, gqla_path path);
+
+/* Cached bytes per token per layer: absorb path (r + d_rope) elements, GQA
+ * path G*(d_nope + d_rope + d_v) elements, times the element size.  At
+ * LLaMA-3-8B shapes the absorb cache is (512+64)/(2*8*128) = 28.125 % of a
+ * GQA baseline with 8 KV heads of 128 ("GQLA" chatpaper.ai Abstract). */
+size_t gqla_cache_bytes_per_token(const gqla_dims* dims, gqla_path path);
+
+/* Static text for a status code. */
+const char* gqla_status_string(gqla_status status);
+
+/* Library version, e.g. "gqla-b200 0.1". */
+const char* gqla_version(void);
+
+/* Number of CUDA kernels this library has launched in this process so far
+ * (all devices, all streams; a diagnostic counter, thread-safe). */
+uint64_t gqla_launch_counter(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQLA_H */

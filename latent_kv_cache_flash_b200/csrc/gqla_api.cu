@@ -1,0 +1,277 @@
+// C-ABI entry points of the GQLA decode library: host-side validation, the
+// split-KV plan, workspace carve-up and kernel dispatch.
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "gqla.h"
+#include "launch.h"
+#include "tc.h"
+
+namespace gqla {
+
+namespace {
+
+constexpr int kSplitGranule = 128;   // token granule of split boundaries
+constexpr int kMaxSplits = 256;
+constexpr int kMinTokensPerSplit = 256;
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+gqla_status check_dims(const gqla_dims* d) {
+  if (!d) return GQLA_ERR_INVALID_ARG;
+  if (d->n_h < 1 || d->G < 1 || d->n_h % d->G != 0) return GQLA_ERR_INVALID_ARG;
+  if (d->d_nope < 1 || d->d_rope < 0 || d->d_v < 1 || d->r < 1) return GQLA_ERR_INVALID_ARG;
+  if (d->s_q < 1 || d->s_q > 4) return GQLA_ERR_INVALID_ARG;
+  if (!(d->scale == d->scale) || isinf(d->scale)) return GQLA_ERR_INVALID_ARG;
+  if (d->dtype != GQLA_F32 && d->dtype != GQLA_BF16) return GQLA_ERR_INVALID_ARG;
+  return GQLA_OK;
+}
+
+gqla_status check_layout(const gqla_kv_layout* l) {
+  if (!l || !l->seq_lens) return GQLA_ERR_INVALID_ARG;
+  if (l->batch < 1 || l->max_seq_len < 1 || l->page_size < 0) return GQLA_ERR_INVALID_ARG;
+  if (l->batch > 65535) return GQLA_ERR_UNSUPPORTED;
+  if (l->page_size == 0) {
+    if (l->capacity < 1) return GQLA_ERR_INVALID_ARG;
+  } else {
+    if (!l->block_table || l->max_blocks_per_seq < 1 || l->num_pages < 1) return GQLA_ERR_INVALID_ARG;
+  }
+  return GQLA_OK;
+}
+
+KvLayout to_kernel_layout(const gqla_kv_layout* l) {
+  KvLayout k;
+  k.seq_lens = l->seq_lens;
+  k.block_table = l->block_table;
+  k.batch = l->batch;
+  k.max_seq_len = l->max_seq_len;
+  k.page_size = l->page_size;
+  k.capacity = l->page_size == 0 ? l->capacity : l->max_blocks_per_seq * l->page_size;
+  k.mbps = l->max_blocks_per_seq;
+  k.num_pages = l->num_pages;
+  return k;
+}
+
+size_t esize(gqla_dtype t) { return t == GQLA_F32 ? 4 : 2; }
+
+SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, gqla_path path) {
+  const int L = l.max_seq_len;
+  int S = requested;
+  if (S <= 0) {
+    // Enough CTAs for two per SM: absorb CTAs cover (sequence, 64-row head
+    // block), GQA CTAs (sequence, group).
+    long long units = path == GQLA_PATH_ABSORB
+                          ? (long long)l.batch * ((d.n_h * d.s_q + 63) / 64)
+                          : (long long)l.batch * d.G;
+    long long want = (2LL * num_sms() + units - 1) / units;
+    long long cap = (L + kMinTokensPerSplit - 1) / kMinTokensPerSplit;
+    S = (int)(want < cap ? want : cap);
+  }
+  if (S < 1) S = 1;
+  if (S > kMaxSplits) S = kMaxSplits;
+  int chunk = (L + S - 1) / S;
+  chunk = ((chunk + kSplitGranule - 1) / kSplitGranule) * kSplitGranule;
+  S = (L + chunk - 1) / chunk;
+  return SplitPlan{S, chunk};
+}
+
+gqla_status make_problem(const gqla_dims* dims, const gqla_kv_layout* layout, int num_splits, gqla_path path,
+                         Problem* p) {
+  gqla_status s = check_dims(dims);
+  if (s != GQLA_OK) return s;
+  s = check_layout(layout);
+  if (s != GQLA_OK) return s;
+  p->d = *dims;
+  p->ly = to_kernel_layout(layout);
+  p->m = dims->n_h / dims->G;
+  p->d_qk = dims->d_nope + dims->d_rope;
+  p->E = dims->r + dims->d_rope;
+  p->rows = (long long)layout->batch * dims->s_q * dims->n_h;
+  p->plan = make_plan(*dims, *layout, num_splits, path);
+  return GQLA_OK;
+}
+
+// The generic kernels keep a row's query and accumulator in registers.
+bool simt_supports(const Problem& p, gqla_path path) {
+  int dk = path == GQLA_PATH_ABSORB ? p.E : p.d_qk;
+  int dv = path == GQLA_PATH_ABSORB ? p.d.r : p.d.d_v;
+  return dk <= 640 && dv <= 512;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+size_t ws_layout(const Problem& p, gqla_path path, bool tc, Workspace* ws, char* base) {
+  size_t off = 0;
+  const int S = p.plan.num_splits;
+  const int D = path == GQLA_PATH_ABSORB ? p.d.r : p.d.d_v;
+  Workspace w{nullptr, nullptr, nullptr, nullptr};
+  if (path == GQLA_PATH_ABSORB) {
+    size_t qt_bytes = (size_t)p.rows * p.d.r * (tc ? 2 : 4);
+    w.qt = base ? base + off : nullptr;
+    off = align256(off + qt_bytes);
+    w.o_lat = base ? (float*)(base + off) : nullptr;
+    off = align256(off + (size_t)p.rows * p.d.r * 4);
+  }
+  if (S > 1) {
+    w.o_part = base ? (float*)(base + off) : nullptr;
+    off = align256(off + (size_t)S * p.rows * D * 4);
+    w.lse_part = base ? (float*)(base + off) : nullptr;
+    off = align256(off + (size_t)S * p.rows * 4);
+  }
+  if (ws) *ws = w;
+  return off;
+}
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+int num_sms() {
+  static std::mutex mu;
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 148;
+  }
+  std::lock_guard<std::mutex> g(mu);
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace gqla
+
+using namespace gqla;
+
+extern "C" {
+
+const char* gqla_version(void) { return "gqla-b200 0.1"; }
+
+uint64_t gqla_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* gqla_status_string(gqla_status s) {
+  switch (s) {
+    case GQLA_OK: return "GQLA_OK";
+    case GQLA_ERR_INVALID_ARG: return "GQLA_ERR_INVALID_ARG: invalid argument";
+    case GQLA_ERR_UNSUPPORTED: return "GQLA_ERR_UNSUPPORTED: dims not handled by this build";
+    case GQLA_ERR_ALIGNMENT: return "GQLA_ERR_ALIGNMENT: pointer or pitch not 16-byte aligned";
+    case GQLA_ERR_WORKSPACE: return "GQLA_ERR_WORKSPACE: workspace missing or too small";
+    case GQLA_ERR_CUDA: return "GQLA_ERR_CUDA: CUDA launch failed";
+  }
+  return "unknown gqla_status";
+}
+
+size_t gqla_cache_bytes_per_token(const gqla_dims* dims, gqla_path path) {
+  if (check_dims(dims) != GQLA_OK) return 0;
+  size_t e = esize(dims->dtype);
+  if (path == GQLA_PATH_ABSORB) return (size_t)(dims->r + dims->d_rope) * e;
+  if (path == GQLA_PATH_GQA) return (size_t)dims->G * (dims->d_nope + dims->d_rope + dims->d_v) * e;
+  return 0;
+}
+
+int32_t gqla_num_splits(const gqla_dims* dims, const gqla_kv_layout* layout, int32_t num_splits, gqla_path path) {
+  Problem p;
+  if (make_problem(dims, layout, num_splits, path, &p) != GQLA_OK) return 0;
+  return p.plan.num_splits;
+}
+
+size_t gqla_workspace_bytes(const gqla_dims* dims, const gqla_kv_layout* layout, int32_t num_splits,
+                            gqla_path path) {
+  Problem p;
+  if (make_problem(dims, layout, num_splits, path, &p) != GQLA_OK) return 0;
+  bool tc = path == GQLA_PATH_ABSORB ? tc_absorb_supports(p) : false;
+  return ws_layout(p, path, tc, nullptr, nullptr);
+}
+
+gqla_status gqla_expand_cache(const gqla_dims* dims, const gqla_kv_layout* layout, const void* latent,
+                              const void* W_uk, const void* W_uv, void* k_pool, void* v_pool,
+                              int32_t tail_tokens, int32_t* dev_status, void* stream) {
+  Problem p;
+  gqla_status s = make_problem(dims, layout, 1, GQLA_PATH_GQA, &p);
+  if (s != GQLA_OK) return s;
+  if (!latent || !W_uk || !W_uv || !k_pool || !v_pool) return GQLA_ERR_INVALID_ARG;
+  if (!aligned16(latent) || !aligned16(W_uk) || !aligned16(W_uv) || !aligned16(k_pool) || !aligned16(v_pool))
+    return GQLA_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (tc_expand_supports(p)) e = tc_expand(p, latent, W_uk, W_uv, k_pool, v_pool, tail_tokens, dev_status, st);
+  else e = simt_expand(p, latent, W_uk, W_uv, k_pool, v_pool, tail_tokens, dev_status, st);
+  return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;
+}
+
+gqla_status gqla_splitkv_combine(int32_t num_splits, int32_t rows, int32_t D, const float* o_part,
+                                 const float* lse_part, void* out, gqla_dtype out_dtype, float* lse_out,
+                                 void* stream) {
+  if (num_splits < 1 || rows < 1 || D < 1 || !o_part || !lse_part || !out) return GQLA_ERR_INVALID_ARG;
+  if (out_dtype != GQLA_F32 && out_dtype != GQLA_BF16) return GQLA_ERR_INVALID_ARG;
+  cudaError_t e = combine(num_splits, rows, D, o_part, lse_part, out, out_dtype, lse_out, (cudaStream_t)stream);
+  return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;
+}
+
+gqla_status gqla_decode_gqa(const gqla_dims* dims, const gqla_kv_layout* layout, const void* q,
+                            const void* k_pool, const void* v_pool, void* out, float* lse, int32_t num_splits,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  Problem p;
+  gqla_status s = make_problem(dims, layout, num_splits, GQLA_PATH_GQA, &p);
+  if (s != GQLA_OK) return s;
+  if (!q || !k_pool || !v_pool || !out) return GQLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out)) return GQLA_ERR_ALIGNMENT;
+  const bool tc = tc_gqa_supports(p);
+  if (!tc && !simt_supports(p, GQLA_PATH_GQA)) return GQLA_ERR_UNSUPPORTED;
+  Workspace w;
+  size_t need = ws_layout(p, GQLA_PATH_GQA, false, &w, (char*)workspace);
+  if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u))) return GQLA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int S = p.plan.num_splits;
+  cudaError_t e;
+  if (tc) e = tc_gqa_decode(p, q, k_pool, v_pool, S > 1 ? nullptr : out, S > 1 ? w.o_part : nullptr,
+                            S > 1 ? w.lse_part : lse, dev_status, st);
+  else e = simt_decode(p, GQLA_PATH_GQA, q, nullptr, k_pool, v_pool, S > 1 ? nullptr : out,
+                       S > 1 ? w.o_part : nullptr, S > 1 ? w.lse_part : lse, dev_status, st);
+  if (e == cudaSuccess && S > 1) e = combine(S, p.rows, p.d.d_v, w.o_part, w.lse_part, out, p.d.dtype, lse, st);
+  return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;
+}
+
+gqla_status gqla_decode_absorb(const gqla_dims* dims, const gqla_kv_layout* layout, const void* q,
+                               const void* latent, const void* W_uk, const void* W_uv, void* out, float* lse,
+                               int32_t num_splits, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                               void* stream) {
+  Problem p;
+  gqla_status s = make_problem(dims, layout, num_splits, GQLA_PATH_ABSORB, &p);
+  if (s != GQLA_OK) return s;
+  if (!q || !latent || !W_uk || !W_uv || !out) return GQLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(latent) || !aligned16(W_uk) || !aligned16(W_uv) || !aligned16(out))
+    return GQLA_ERR_ALIGNMENT;
+  const bool tc = tc_absorb_supports(p);
+  if (!tc && !simt_supports(p, GQLA_PATH_ABSORB)) return GQLA_ERR_UNSUPPORTED;
+  Workspace w;
+  size_t need = ws_layout(p, GQLA_PATH_ABSORB, tc, &w, (char*)workspace);
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)) return GQLA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int S = p.plan.num_splits;
+  cudaError_t e;
+  if (tc) {
+    e = tc_absorb_decode(p, q, latent, W_uk, W_uv, out, lse, w, dev_status, st);
+  } else {
+    e = simt_absorb_q(p, q, W_uk, (float*)w.qt, st);
+    if (e == cudaSuccess)
+      e = simt_decode(p, GQLA_PATH_ABSORB, q, (const float*)w.qt, latent, latent, nullptr,
+                      S > 1 ? w.o_part : w.o_lat, S > 1 ? w.lse_part : lse, dev_status, st);
+    if (e == cudaSuccess && S > 1) e = combine(S, p.rows, p.d.r, w.o_part, w.lse_part, w.o_lat, GQLA_F32, lse, st);
+    if (e == cudaSuccess) e = simt_up_proj(p, w.o_lat, W_uv, out, st);
+  }
+  return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;
+}
+
+}  // extern "C"

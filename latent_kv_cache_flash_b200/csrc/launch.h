@@ -1,0 +1,57 @@
+// Host-side launchers shared between the API translation unit and the kernel
+// translation units of the GQLA library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "gqla.h"
+
+namespace gqla {
+
+// A validated decode problem with the derived sizes.
+struct Problem {
+  gqla_dims d;
+  KvLayout ly;
+  int m;        // heads per group
+  int d_qk;     // d_nope + d_rope
+  int E;        // latent row width r + d_rope
+  long long rows;  // B * s_q * n_h output rows
+  SplitPlan plan;
+};
+
+// Workspace carve-up of one decode call (all fp32 except qt, which is fp32 for
+// the SIMT path and bf16 for the tensor-core path).
+struct Workspace {
+  void* qt;        // absorbed queries [rows, r]
+  float* o_part;   // [S, rows, D] when S > 1
+  float* lse_part; // [S, rows] when S > 1
+  float* o_lat;    // absorb: combined latent outputs [rows, r]
+};
+
+size_t ws_layout(const Problem& p, gqla_path path, bool tc, Workspace* ws, char* base);
+
+// ---- generic CUDA-core kernels (fp32 math; any supported dims) ----
+cudaError_t simt_expand(const Problem& p, const void* latent, const void* W_uk, const void* W_uv,
+                        void* k_pool, void* v_pool, int tail, int32_t* st, cudaStream_t s);
+cudaError_t simt_absorb_q(const Problem& p, const void* q, const void* W_uk, float* qt,
+                          cudaStream_t s);
+// path GQA: keys/values are the expanded pools; path ABSORB: the latent pool.
+// Writes o (normalised) + lse per (split, row): to o_part/lse_part when S > 1,
+// else to out_T (GQA) or o_lat (absorb) and lse.
+cudaError_t simt_decode(const Problem& p, gqla_path path, const void* q, const float* qt,
+                        const void* kpool, const void* vpool, void* out_T, float* o_f32,
+                        float* lse, int32_t* st, cudaStream_t s);
+cudaError_t simt_up_proj(const Problem& p, const float* o_lat, const void* W_uv, void* out,
+                         cudaStream_t s);
+cudaError_t combine(int S, long long rows, int D, const float* o_part, const float* lse_part,
+                    void* out, gqla_dtype out_dtype, float* lse_out, cudaStream_t s);
+
+int num_sms();
+
+// Counts one kernel launch (reported by gqla_launch_counter).
+void count_launch(int n = 1);
+
+}  // namespace gqla

@@ -1,0 +1,26 @@
+// Tensor-core (bf16) kernels of the GQLA decode library.
+#pragma once
+
+#include "launch.h"
+
+namespace gqla {
+
+// GQA decode over the expanded cache: mma.sync bf16 tiles, cp.async.bulk
+// staged K/V pages, online softmax per 16-row block.
+bool tc_gqa_supports(const Problem& p);
+cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
+                          float* o_part, float* lse_dst, int32_t* st, cudaStream_t s);
+
+// MQA-absorb decode: absorbed query, latent attention on tcgen05/TMEM, combine,
+// up-projection.
+bool tc_absorb_supports(const Problem& p);
+cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent, const void* W_uk,
+                             const void* W_uv, void* out, float* lse, const Workspace& w, int32_t* st,
+                             cudaStream_t s);
+
+// Cache expansion GEMM on tcgen05.
+bool tc_expand_supports(const Problem& p);
+cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, const void* W_uv, void* k_pool,
+                      void* v_pool, int tail, int32_t* st, cudaStream_t s);
+
+}  // namespace gqla

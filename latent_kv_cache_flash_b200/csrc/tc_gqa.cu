@@ -1,0 +1,379 @@
+// GQA-path decode over the per-group expanded cache, bf16, on sm_100a.
+//
+// Grouped-query decode ("GQLA" chatpaper.ai Abstract: a GQA path with a
+// per-group expanded cache; "Grouped Query Attention (GQA)" glossary,
+// "Fonctionnement de la GQA": every query head of group g attends over the
+// group's single K/V head).  Decode at m*s_q <= 16 rows per group is a
+// bandwidth-bound stream of the K/V pages (640 bytes per group-token at
+// d_qk = 192, d_v = 128), so the kernel is built around moving those bytes:
+//
+//  * one CTA per (key-range split, sequence, group[, 64-row block]);
+//  * a producer warp streams 64-token K and V tiles with TMA (3-D tensor maps
+//    over the pool's [token row, group, dim] view, 128-byte swizzle) into a
+//    2-stage mbarrier ring; two CTAs fit on an SM;
+//  * four consumer warps each take 16 tokens of a tile (or, for more than 16
+//    rows, one 16-row block each), compute S = Q K^T and O += P V with
+//    mma.sync m16n8k16 bf16 (fp32 accumulate) from ldmatrix'd fragments, and
+//    keep an online softmax (running max in the log2 domain) per row;
+//  * the warps' partial states are merged through shared memory at the end;
+//    the result goes to `out` (one split) or to fp32 split partials.
+#include <math.h>
+
+#include "ptx.cuh"
+#include "tc.h"
+
+namespace gqla {
+
+namespace {
+
+constexpr int kDqk = 192;
+constexpr int kDv = 128;
+constexpr int kT = 64;                       // tokens per tile
+constexpr int kStages = 2;
+constexpr int kKChunks = kDqk / 64;          // 64-column (128-byte) chunks
+constexpr int kVChunks = kDv / 64;
+constexpr int kChunkBytes = kT * 128;
+constexpr int kStageBytes = (kKChunks + kVChunks) * kChunkBytes;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kOStride = kDv + 4;            // merge buffer row pitch (floats)
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024;
+
+struct GqaParams {
+  KvLayout ly;
+  SplitPlan plan;
+  const __nv_bfloat16* q;
+  __nv_bfloat16* out;
+  float* o_part;
+  float* lse;
+  int n_h, G, m, s_q;
+  int rows_unit;   // m * s_q rows of one (sequence, group)
+  int rbc;         // 16-row blocks per CTA: 1, 2 or 4
+  float scale_log2;
+  long long rows;  // B * s_q * n_h
+  int32_t* st;
+};
+
+static_assert(kConsumerWarps * 16 * kOStride * 4 + 2 * kConsumerWarps * 16 * 4 <= kStages * kStageBytes,
+              "merge buffer must fit in the stage ring");
+
+__global__ void __launch_bounds__(kThreads, 2)
+    gqa_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                      const GqaParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x;
+  const int b = blockIdx.y / p.G, g = blockIdx.y % p.G;
+  const int rb0 = blockIdx.z * p.rbc;            // first global 16-row block of this CTA
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(&full_bar[s], 1);
+      ptx::mbar_init(&empty_bar[s], kConsumerWarps);
+    }
+    abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  int L = seq_len_checked(p.ly, b, p.s_q, (split == 0 && g == 0 && blockIdx.z == 0) ? p.st : nullptr);
+  if (!seq_pages_ok(p.ly, b, L, p.st)) L = -1;   // includes a __syncthreads
+  const int t_begin = split * p.plan.chunk;
+  const int t_stop = L < 0 ? t_begin : min(t_begin + p.plan.chunk, L);
+  const int n_tiles = t_stop > t_begin ? (t_stop - t_begin + kT - 1) / kT : 0;
+
+  if (warp == kConsumerWarps) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&kmap);
+      ptx::prefetch_tmap(&vmap);
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % kStages, k = j / kStages;
+        if (k > 0 && !ptx::mbar_wait(&empty_bar[s], (k - 1) & 1)) {
+          flag_status(p.st, GQLA_DEV_TIMEOUT);
+          atomicExch(&abort_flag, 1);
+          break;
+        }
+        if (*(volatile int*)&abort_flag) break;
+        const int t0 = t_begin + j * kT;
+        const int row0 = (int)token_row(p.ly, b, t0, nullptr);
+        uint8_t* st = smem + s * kStageBytes;
+        ptx::mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
+#pragma unroll
+        for (int c = 0; c < kKChunks; ++c) ptx::tma_load_3d(st + c * kChunkBytes, &kmap, &full_bar[s], 64 * c, g, row0);
+#pragma unroll
+        for (int c = 0; c < kVChunks; ++c)
+          ptx::tma_load_3d(st + (kKChunks + c) * kChunkBytes, &vmap, &full_bar[s], 64 * c, g, row0);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int ts = kConsumerWarps / p.rbc;         // token slices per tile
+  const int rbl = warp / ts, slice = warp % ts;
+  const int sub_steps = (kT / ts) / 16;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int rbg = rb0 + rbl;                      // this warp's global row block
+  int vis[2];
+  long long grow[2];
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const int r = rbg * 16 + gid + 8 * h2;
+    if (r < p.rows_unit && L >= 0) {
+      const int i = r / p.m, h = g * p.m + r % p.m;
+      vis[h2] = L - p.s_q + i + 1;
+      grow[h2] = ((long long)b * p.s_q + i) * p.n_h + h;
+    } else {
+      vis[h2] = 0;
+      grow[h2] = -1;
+    }
+  }
+  // Q fragments (A operand, 16 rows x 192) straight from global memory.
+  uint32_t qa[kDqk / 16][4];
+#pragma unroll
+  for (int kk = 0; kk < kDqk / 16; ++kk) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int h2 = e & 1, hi = e >> 1;
+      uint32_t v = 0;
+      if (grow[h2] >= 0)
+        v = *reinterpret_cast<const uint32_t*>(p.q + grow[h2] * kDqk + kk * 16 + hi * 8 + 2 * tig);
+      qa[kk][e] = v;
+    }
+  }
+  float o[kDv / 8][4];
+#pragma unroll
+  for (int n = 0; n < kDv / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  bool aborted = false;
+
+  for (int j = 0; j < n_tiles; ++j) {
+    const int s = j % kStages;
+    if (!ptx::mbar_wait(&full_bar[s], (j / kStages) & 1)) {
+      flag_status(p.st, GQLA_DEV_TIMEOUT);
+      atomicExch(&abort_flag, 1);
+      aborted = true;
+      break;
+    }
+    const int t0 = t_begin + j * kT;
+    const uint8_t* st = smem + s * kStageBytes;
+    const uint32_t kbase = ptx::smem_u32(st);
+    const uint32_t vbase = kbase + kKChunks * kChunkBytes;
+    if (t0 + kT > L) {
+      // rows past the sequence may hold anything: zero this warp's V rows there
+      for (int idx = lane; idx < (kT / ts) * kVChunks * 8; idx += 32) {
+        const int tok = slice * (kT / ts) + idx / (kVChunks * 8);
+        const int rem = idx % (kVChunks * 8);
+        if (t0 + tok >= L)
+          *reinterpret_cast<uint4*>(const_cast<uint8_t*>(st) + kKChunks * kChunkBytes + (rem / 8) * kChunkBytes +
+                                    ptx::swz128(tok, rem % 8)) = make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
+    for (int u = 0; u < sub_steps; ++u) {
+      const int tt0 = slice * (kT / ts) + u * 16;
+      float sc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sc[e] = 0.f;
+      const int mat = lane >> 3, mr = lane & 7;
+#pragma unroll
+      for (int kk = 0; kk < kDqk / 16; ++kk) {
+        const int tok = tt0 + (mat >> 1) * 8 + mr;
+        const int gi = (kk & 3) * 2 + (mat & 1);
+        uint32_t r0, r1, r2, r3;
+        ptx::ldsm_x4(kbase + (kk >> 2) * kChunkBytes + ptx::swz128(tok, gi), r0, r1, r2, r3);
+        ptx::mma_bf16_16816(&sc[0], qa[kk], r0, r1);
+        ptx::mma_bf16_16816(&sc[4], qa[kk], r2, r3);
+      }
+      // scale into the log2 domain and mask invisible tokens (select, so a
+      // non-finite key past the end cannot leak in)
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int h2 = (e >> 1) & 1;
+        const int tok = t0 + tt0 + (e >> 2) * 8 + 2 * tig + (e & 1);
+        sc[e] = tok < vis[h2] ? sc[e] * p.scale_log2 : -INFINITY;
+        mx[h2] = fmaxf(mx[h2], sc[e]);
+      }
+      float corr[2];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 1));
+        mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 2));
+        const float mn = fmaxf(mrow[h2], mx[h2]);
+        corr[h2] = mn == -INFINITY ? 1.f : ptx::fast_exp2(mrow[h2] - mn);
+        mrow[h2] = mn;
+      }
+      float ps[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int h2 = (e >> 1) & 1;
+        ps[e] = mrow[h2] == -INFINITY ? 0.f : ptx::fast_exp2(sc[e] - mrow[h2]);
+      }
+      lrow[0] = lrow[0] * corr[0] + (ps[0] + ps[1] + ps[4] + ps[5]);
+      lrow[1] = lrow[1] * corr[1] + (ps[2] + ps[3] + ps[6] + ps[7]);
+      if (corr[0] != 1.f || corr[1] != 1.f) {
+#pragma unroll
+        for (int n = 0; n < kDv / 8; ++n) {
+          o[n][0] *= corr[0];
+          o[n][1] *= corr[0];
+          o[n][2] *= corr[1];
+          o[n][3] *= corr[1];
+        }
+      }
+      uint32_t pa[4];
+      pa[0] = ptx::pack_bf16(ps[0], ps[1]);
+      pa[1] = ptx::pack_bf16(ps[2], ps[3]);
+      pa[2] = ptx::pack_bf16(ps[4], ps[5]);
+      pa[3] = ptx::pack_bf16(ps[6], ps[7]);
+#pragma unroll
+      for (int np = 0; np < kDv / 16; ++np) {
+        const int tok = tt0 + (mat & 1) * 8 + mr;
+        const int gi = (np & 3) * 2 + (mat >> 1);
+        uint32_t r0, r1, r2, r3;
+        ptx::ldsm_x4_t(vbase + (np >> 2) * kChunkBytes + ptx::swz128(tok, gi), r0, r1, r2, r3);
+        ptx::mma_bf16_16816(o[2 * np], pa, r0, r1);
+        ptx::mma_bf16_16816(o[2 * np + 1], pa, r2, r3);
+      }
+    }
+    if (t0 + kT > L) ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty_bar[s]);
+  }
+
+  // ------------------------------------------------ merge the token slices
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    lrow[h2] += __shfl_xor_sync(0xffffffffu, lrow[h2], 1);
+    lrow[h2] += __shfl_xor_sync(0xffffffffu, lrow[h2], 2);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+  if (aborted || *(volatile int*)&abort_flag) return;
+  float* ob = reinterpret_cast<float*>(smem);                       // [warp][16][kOStride]
+  float* ml = ob + kConsumerWarps * 16 * kOStride;                  // [warp][16] max, then [warp][16] sum
+#pragma unroll
+  for (int n = 0; n < kDv / 8; ++n) {
+    *reinterpret_cast<float2*>(&ob[(warp * 16 + gid) * kOStride + n * 8 + 2 * tig]) = make_float2(o[n][0], o[n][1]);
+    *reinterpret_cast<float2*>(&ob[(warp * 16 + gid + 8) * kOStride + n * 8 + 2 * tig]) =
+        make_float2(o[n][2], o[n][3]);
+  }
+  if (tig == 0) {
+    ml[warp * 16 + gid] = mrow[0];
+    ml[warp * 16 + gid + 8] = mrow[1];
+    ml[kConsumerWarps * 16 + warp * 16 + gid] = lrow[0];
+    ml[kConsumerWarps * 16 + warp * 16 + gid + 8] = lrow[1];
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+  // each warp finishes 16 / ts rows of its row block
+  const int rows_per = 16 / ts;
+  for (int rr = slice * rows_per; rr < (slice + 1) * rows_per; ++rr) {
+    const int r = (rb0 + rbl) * 16 + rr;
+    if (r >= p.rows_unit) break;
+    const int i = r / p.m, h = g * p.m + r % p.m;
+    const long long gr = ((long long)b * p.s_q + i) * p.n_h + h;
+    float mt = -INFINITY;
+    for (int w = 0; w < ts; ++w) mt = fmaxf(mt, ml[(rbl * ts + w) * 16 + rr]);
+    float wsum = 0.f, wgt[kConsumerWarps];
+    for (int w = 0; w < ts; ++w) {
+      const float mw = ml[(rbl * ts + w) * 16 + rr];
+      wgt[w] = mw == -INFINITY ? 0.f : ptx::fast_exp2(mw - mt);
+      wsum += wgt[w] * ml[kConsumerWarps * 16 + (rbl * ts + w) * 16 + rr];
+    }
+    const bool empty = !(wsum > 0.f);
+    const float inv = empty ? 0.f : 1.f / wsum;
+    for (int d = lane; d < kDv; d += 32) {
+      float acc = 0.f;
+      for (int w = 0; w < ts; ++w) acc += wgt[w] * ob[((rbl * ts + w) * 16 + rr) * kOStride + d];
+      acc *= inv;
+      if (p.o_part) p.o_part[((long long)split * p.rows + gr) * kDv + d] = acc;
+      else p.out[gr * kDv + d] = __float2bfloat16_rn(acc);
+    }
+    if (lane == 0 && p.lse) {
+      const float lse = empty ? -INFINITY : (mt + log2f(wsum)) * 0.69314718055994531f;
+      p.lse[p.o_part ? (long long)split * p.rows + gr : gr] = lse;
+    }
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)f;
+  }
+  return fn;
+}
+
+// [dim (inner), group, token row] view of a per-group pool, 64x1x64 boxes.
+bool make_pool_map(CUtensorMap* map, const void* base, int dim, int G, long long nrows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3] = {(cuuint64_t)dim, (cuuint64_t)G, (cuuint64_t)nrows};
+  cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * 2 * G};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kT};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tc_gqa_supports(const Problem& p) {
+  const auto& d = p.d;
+  if (d.dtype != GQLA_BF16) return false;
+  if (p.d_qk != kDqk || d.d_v != kDv) return false;
+  if (p.ly.page_size != 0 && p.ly.page_size % kT != 0) return false;
+  if ((long long)p.ly.batch * d.G > 65535) return false;
+  return true;
+}
+
+cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
+                          float* o_part, float* lse_dst, int32_t* st, cudaStream_t s) {
+  const auto& d = p.d;
+  long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
+                                        : (long long)p.ly.num_pages * p.ly.page_size;
+  CUtensorMap kmap, vmap;
+  if (!make_pool_map(&kmap, k_pool, kDqk, d.G, nrows) || !make_pool_map(&vmap, v_pool, kDv, d.G, nrows))
+    return cudaErrorInvalidValue;
+  GqaParams prm;
+  prm.ly = p.ly;
+  prm.plan = p.plan;
+  prm.q = (const __nv_bfloat16*)q;
+  prm.out = (__nv_bfloat16*)out;
+  prm.o_part = o_part;
+  prm.lse = lse_dst;
+  prm.n_h = d.n_h;
+  prm.G = d.G;
+  prm.m = p.m;
+  prm.s_q = d.s_q;
+  prm.rows_unit = p.m * d.s_q;
+  const int rb = (prm.rows_unit + 15) / 16;
+  prm.rbc = rb >= 4 ? 4 : (rb == 3 ? 4 : rb);
+  prm.scale_log2 = d.scale * 1.4426950408889634f;
+  prm.rows = p.rows;
+  prm.st = st;
+  dim3 grid(p.plan.num_splits, p.ly.batch * d.G, (rb + prm.rbc - 1) / prm.rbc);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(gqa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    attr = true;
+  }
+  gqa_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace gqla

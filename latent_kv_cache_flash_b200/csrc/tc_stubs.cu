@@ -1,0 +1,23 @@
+// Placeholders for tensor-core kernels not built yet: every problem goes to
+// the generic kernels.
+#include "tc.h"
+
+namespace gqla {
+
+bool tc_gqa_supports(const Problem&) { return false; }
+cudaError_t tc_gqa_decode(const Problem&, const void*, const void*, const void*, void*, float*, float*, int32_t*,
+                          cudaStream_t) {
+  return cudaErrorNotSupported;
+}
+bool tc_absorb_supports(const Problem&) { return false; }
+cudaError_t tc_absorb_decode(const Problem&, const void*, const void*, const void*, const void*, void*, float*,
+                             const Workspace&, int32_t*, cudaStream_t) {
+  return cudaErrorNotSupported;
+}
+bool tc_expand_supports(const Problem&) { return false; }
+cudaError_t tc_expand(const Problem&, const void*, const void*, const void*, void*, void*, int, int32_t*,
+                      cudaStream_t) {
+  return cudaErrorNotSupported;
+}
+
+}  // namespace gqla

@@ -1,0 +1,174 @@
+"""ctypes binding of libgqla.so (declared in include/gqla.h).
+
+Argument marshalling only: every step of the decode path runs in the
+library's CUDA kernels.  torch tensors supply device pointers, the current
+CUDA stream and, when the caller passes none, the workspace buffer.  The
+functions keep the C names; a non-OK status raises :class:`GqlaError`.
+There is no fallback: if the library is missing, loading raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqla.so")
+
+GQLA_OK, GQLA_ERR_INVALID_ARG, GQLA_ERR_UNSUPPORTED, GQLA_ERR_ALIGNMENT, GQLA_ERR_WORKSPACE, GQLA_ERR_CUDA = range(6)
+GQLA_F32, GQLA_BF16 = 0, 1
+GQLA_PATH_ABSORB, GQLA_PATH_GQA = 0, 1
+DEV_SHORT_SEQ, DEV_OVERFLOW, DEV_BAD_PAGE, DEV_TIMEOUT = 1, 2, 4, 8
+
+
+class GqlaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+class GqlaDims(ctypes.Structure):
+    _fields_ = [("n_h", ctypes.c_int32), ("G", ctypes.c_int32), ("d_nope", ctypes.c_int32),
+                ("d_rope", ctypes.c_int32), ("d_v", ctypes.c_int32), ("r", ctypes.c_int32),
+                ("s_q", ctypes.c_int32), ("scale", ctypes.c_float), ("dtype", ctypes.c_int)]
+
+
+class GqlaKvLayout(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("seq_lens", ctypes.c_void_p), ("max_seq_len", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("capacity", ctypes.c_int32), ("block_table", ctypes.c_void_p),
+                ("max_blocks_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """Loads libgqla.so once; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError("libgqla.so not built: run python -m latent_kv_cache_flash_b200.build")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        pd, pl = ctypes.POINTER(GqlaDims), ctypes.POINTER(GqlaKvLayout)
+        L.gqla_expand_cache.argtypes = [pd, pl, P, P, P, P, P, I32, P, P]
+        L.gqla_decode_absorb.argtypes = [pd, pl, P, P, P, P, P, P, I32, P, SZ, P, P]
+        L.gqla_decode_gqa.argtypes = [pd, pl, P, P, P, P, P, I32, P, SZ, P, P]
+        L.gqla_splitkv_combine.argtypes = [I32, I32, I32, P, P, P, ctypes.c_int, P, P]
+        L.gqla_workspace_bytes.argtypes = [pd, pl, I32, ctypes.c_int]
+        L.gqla_workspace_bytes.restype = SZ
+        L.gqla_num_splits.argtypes = [pd, pl, I32, ctypes.c_int]
+        L.gqla_num_splits.restype = I32
+        L.gqla_cache_bytes_per_token.argtypes = [pd, ctypes.c_int]
+        L.gqla_cache_bytes_per_token.restype = SZ
+        L.gqla_status_string.argtypes = [ctypes.c_int]
+        L.gqla_status_string.restype = ctypes.c_char_p
+        L.gqla_version.restype = ctypes.c_char_p
+        L.gqla_launch_counter.restype = ctypes.c_uint64
+        for name in ("gqla_expand_cache", "gqla_decode_absorb", "gqla_decode_gqa", "gqla_splitkv_combine"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is not None:
+        return ctypes.c_void_p(stream)
+    if device is not None and device.type == "cuda":
+        return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    return None
+
+
+def _check(status: int, what: str):
+    if status != GQLA_OK:
+        raise GqlaError(status, "%s: %s" % (what, gqla_status_string(status)))
+
+
+def make_dims(d) -> GqlaDims:
+    """Builds the C struct from any object with n_h, G, d_nope, d_rope, d_v, r,
+    s_q, softmax_scale (or scale) and dtype ("f32"/"bf16")."""
+    scale = getattr(d, "softmax_scale", None)
+    if scale is None:
+        scale = d.scale
+    dt = GQLA_F32 if d.dtype in ("f32", torch.float32) else GQLA_BF16
+    return GqlaDims(d.n_h, d.G, d.d_nope, d.d_rope, d.d_v, d.r, d.s_q, float(scale), dt)
+
+
+def make_layout(seq_lens: torch.Tensor, max_seq_len: int, page_size: int = 0, capacity: int = 0,
+                block_table: Optional[torch.Tensor] = None, num_pages: int = 0) -> GqlaKvLayout:
+    """seq_lens and block_table are int32 device tensors (kept alive by the caller)."""
+    mbps = 0 if block_table is None else int(block_table.shape[1])
+    return GqlaKvLayout(int(seq_lens.shape[0]), _ptr(seq_lens), int(max_seq_len), int(page_size),
+                        int(capacity), _ptr(block_table), mbps, int(num_pages))
+
+
+def gqla_status_string(status: int) -> str:
+    return lib().gqla_status_string(status).decode()
+
+
+def gqla_version() -> str:
+    return lib().gqla_version().decode()
+
+
+def gqla_launch_counter() -> int:
+    return int(lib().gqla_launch_counter())
+
+
+def gqla_cache_bytes_per_token(dims: GqlaDims, path: int) -> int:
+    return int(lib().gqla_cache_bytes_per_token(ctypes.byref(dims), path))
+
+
+def gqla_workspace_bytes(dims: GqlaDims, layout: GqlaKvLayout, num_splits: int, path: int) -> int:
+    return int(lib().gqla_workspace_bytes(ctypes.byref(dims), ctypes.byref(layout), num_splits, path))
+
+
+def gqla_num_splits(dims: GqlaDims, layout: GqlaKvLayout, num_splits: int, path: int) -> int:
+    return int(lib().gqla_num_splits(ctypes.byref(dims), ctypes.byref(layout), num_splits, path))
+
+
+def workspace_for(dims: GqlaDims, layout: GqlaKvLayout, num_splits: int, path: int, device) -> torch.Tensor:
+    n = gqla_workspace_bytes(dims, layout, num_splits, path)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def gqla_expand_cache(dims, layout, latent, W_uk, W_uv, k_pool, v_pool, tail_tokens=0, dev_status=None,
+                      stream=None):
+    s = lib().gqla_expand_cache(ctypes.byref(dims), ctypes.byref(layout), _ptr(latent), _ptr(W_uk), _ptr(W_uv),
+                                _ptr(k_pool), _ptr(v_pool), int(tail_tokens), _ptr(dev_status),
+                                _stream(stream, latent.device))
+    _check(s, "gqla_expand_cache")
+
+
+def gqla_decode_absorb(dims, layout, q, latent, W_uk, W_uv, out, lse=None, num_splits=0, workspace=None,
+                       dev_status=None, stream=None):
+    if workspace is None:
+        workspace = workspace_for(dims, layout, num_splits, GQLA_PATH_ABSORB, q.device)
+    s = lib().gqla_decode_absorb(ctypes.byref(dims), ctypes.byref(layout), _ptr(q), _ptr(latent), _ptr(W_uk),
+                                 _ptr(W_uv), _ptr(out), _ptr(lse), int(num_splits), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                 _stream(stream, q.device))
+    _check(s, "gqla_decode_absorb")
+
+
+def gqla_decode_gqa(dims, layout, q, k_pool, v_pool, out, lse=None, num_splits=0, workspace=None,
+                    dev_status=None, stream=None):
+    if workspace is None:
+        workspace = workspace_for(dims, layout, num_splits, GQLA_PATH_GQA, q.device)
+    s = lib().gqla_decode_gqa(ctypes.byref(dims), ctypes.byref(layout), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                              _ptr(out), _ptr(lse), int(num_splits), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                              _stream(stream, q.device))
+    _check(s, "gqla_decode_gqa")
+
+
+def gqla_splitkv_combine(o_part, lse_part, out, lse_out=None, stream=None):
+    S, rows, D = (int(x) for x in o_part.shape)
+    dt = GQLA_F32 if out.dtype == torch.float32 else GQLA_BF16
+    s = lib().gqla_splitkv_combine(S, rows, D, _ptr(o_part), _ptr(lse_part), _ptr(out), dt, _ptr(lse_out),
+                                   _stream(stream, o_part.device))
+    _check(s, "gqla_splitkv_combine")

@@ -1,0 +1,126 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports
+every function include/gqla.h declares, validates arguments before launching
+anything, and its size helpers agree with the page figures."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def G():
+    from latent_kv_cache_flash_b200 import build, gqla
+    build.build()
+    return gqla
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "gqla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gqla_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(G):
+    names = declared_functions()
+    assert len(names) >= 9
+    lib = G.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert G.gqla_version().startswith("gqla-b200")
+
+
+def test_status_strings(G):
+    for s in range(6):
+        assert G.gqla_status_string(s).startswith("GQLA_")
+
+
+def _dims(mod, **kw):
+    base = dict(n_h=32, G=8, d_nope=128, d_rope=64, d_v=128, r=512, s_q=1, scale=192 ** -0.5, dtype=mod.GQLA_BF16)
+    base.update(kw)
+    return mod.GqlaDims(*[base[k] for k in ("n_h", "G", "d_nope", "d_rope", "d_v", "r", "s_q", "scale", "dtype")])
+
+
+def _layout(G, B=4, L=8192, page=0):
+    lens = torch.full((B,), L, dtype=torch.int32)
+    return lens, G.GqlaKvLayout(B, lens.data_ptr(), L, page, L if page == 0 else 0,
+                                None if page == 0 else lens.data_ptr(), 1 if page else 0, 1 if page else 0)
+
+
+def test_cache_bytes_28_125_percent(G):
+    gold = json.load(open(os.path.join(ROOT, "tests", "golden", "page_figures.json")))
+    a = gold["absorb_cache_fraction_llama3_8b"]
+    d = _dims(G)
+    absorb = G.gqla_cache_bytes_per_token(d, G.GQLA_PATH_ABSORB)
+    baseline = 2 * a["n_kv_heads"] * a["head_dim"] * 2
+    assert absorb / baseline == a["value"]
+    # the expanded GQLA cache of the same layer: 8 groups * (192 + 128) bf16
+    assert G.gqla_cache_bytes_per_token(d, G.GQLA_PATH_GQA) == 8 * 320 * 2
+
+
+def test_validation_before_launch(G):
+    lens, lay = _layout(G)
+    null = ctypes.c_void_p(0)
+    bad_groups = _dims(G, G=5)
+    L = G.lib()
+    s = L.gqla_decode_gqa(ctypes.byref(bad_groups), ctypes.byref(lay), null, null, null, null, None, 0, null, 0,
+                          None, None)
+    assert s == G.GQLA_ERR_INVALID_ARG
+    d = _dims(G, s_q=5)
+    assert L.gqla_decode_absorb(ctypes.byref(d), ctypes.byref(lay), null, null, null, null, null, None, 0, null,
+                                0, None, None) == G.GQLA_ERR_INVALID_ARG
+    d = _dims(G)
+    # null tensor pointers
+    assert L.gqla_decode_gqa(ctypes.byref(d), ctypes.byref(lay), null, null, null, null, None, 0, null, 0,
+                             None, None) == G.GQLA_ERR_INVALID_ARG
+    # misaligned pointers are refused before any launch
+    p = ctypes.c_void_p(0x1008)
+    assert L.gqla_decode_gqa(ctypes.byref(d), ctypes.byref(lay), p, p, p, p, None, 0, null, 0, None,
+                             None) == G.GQLA_ERR_ALIGNMENT
+    # workspace too small (4 splits requested)
+    a = ctypes.c_void_p(0x10000)
+    assert L.gqla_decode_gqa(ctypes.byref(d), ctypes.byref(lay), a, a, a, a, None, 4, a, 16, None,
+                             None) == G.GQLA_ERR_WORKSPACE
+    # paged layout without a block table
+    bad = G.GqlaKvLayout(4, lens.data_ptr(), 8192, 64, 0, None, 0, 0)
+    assert L.gqla_decode_gqa(ctypes.byref(d), ctypes.byref(bad), a, a, a, a, None, 0, a, 1 << 30, None,
+                             None) == G.GQLA_ERR_INVALID_ARG
+    assert L.gqla_splitkv_combine(0, 4, 8, a, a, a, 0, None, None) == G.GQLA_ERR_INVALID_ARG
+
+
+def test_split_plan_and_workspace(G):
+    lens, lay = _layout(G, B=32, L=8192)
+    d = _dims(G)
+    for req in (1, 2, 3, 8, 64):
+        S = G.gqla_num_splits(d, lay, req, G.GQLA_PATH_GQA)
+        assert 1 <= S <= req
+        chunk = -(-8192 // S)
+        assert S * chunk >= 8192
+    S = G.gqla_num_splits(d, lay, 4, G.GQLA_PATH_GQA)
+    rows = 32 * 1 * 32
+    ws = G.gqla_workspace_bytes(d, lay, 4, G.GQLA_PATH_GQA)
+    assert ws >= S * rows * 128 * 4 + S * rows * 4
+    assert G.gqla_workspace_bytes(d, lay, 1, G.GQLA_PATH_GQA) == 0
+    # auto choice is stable between the two helpers
+    S0 = G.gqla_num_splits(d, lay, 0, G.GQLA_PATH_GQA)
+    assert S0 >= 1
+    assert G.gqla_workspace_bytes(d, lay, 0, G.GQLA_PATH_GQA) == G.gqla_workspace_bytes(d, lay, S0, G.GQLA_PATH_GQA)
+    # absorb always needs the absorbed queries and the latent outputs
+    assert G.gqla_workspace_bytes(d, lay, 1, G.GQLA_PATH_ABSORB) >= rows * 512 * 2 + rows * 512 * 4
+
+
+def test_binding_has_c_names(G):
+    for n in declared_functions():
+        assert hasattr(G, n), n
+
+
+def test_no_cpu_fallback_when_library_missing(tmp_path, monkeypatch):
+    from latent_kv_cache_flash_b200 import gqla
+    monkeypatch.setattr(gqla, "_LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(gqla, "_lib", None)
+    with pytest.raises(ImportError):
+        gqla.lib()

@@ -1,0 +1,240 @@
+"""GPU parity: the CUDA path (through the C-ABI binding) against the fp64
+oracle on the same seeded inputs, plus structural invariances and edge cases.
+
+Tolerances: fp32 max|err| <= 1e-5 max|ref|; bf16 max|err| <= 1e-2 max|ref| +
+1e-3 (fp32 accumulation), applied to the output and to the log-sum-exp."""
+import numpy as np
+import pytest
+import torch
+
+from latent_kv_cache_flash_b200 import synth
+from oracle import gqla_oracle as O
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from latent_kv_cache_flash_b200 import build
+    build.build()
+
+
+def _wl(dims, B, lens, page=0, seed=0):
+    wl = synth.Workload("t", dims, batch=B, seq_len=max(lens), page_size=page, seed=seed)
+    return synth.make_inputs(wl, DEV, seq_lens=lens)
+
+
+LLAMA = dict(n_h=32, G=8, d_nope=128, d_rope=64, d_v=128, r=512)
+DSV3 = dict(n_h=128, G=16, d_nope=128, d_rope=64, d_v=128, r=512)
+
+
+# ---- the tiny fp32 workload, whole output, both paths ----------------------
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+def test_tiny_f32_full(path):
+    inp = synth.make_inputs(synth.tiny_f32(), DEV)
+    out, lse = H.run_decode(inp, path)
+    H.check_units(inp, out, lse, H.all_units(inp), "tiny_f32 " + path)
+
+
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+@pytest.mark.parametrize("splits", [1, 2, 5])
+def test_f32_ragged_splits(path, splits):
+    d = synth.Dims(n_h=8, G=2, d_nope=32, d_rope=16, d_v=32, r=64, s_q=2, dtype="f32")
+    inp = _wl(d, 3, [2, 301, 700])
+    out, lse = H.run_decode(inp, path, num_splits=splits)
+    H.check_units(inp, out, lse, H.all_units(inp), "f32 ragged %s S=%d" % (path, splits))
+
+
+# ---- bf16, LLaMA-3-8B and DeepSeek-V3 head shapes at short contexts --------
+@pytest.mark.parametrize("s_q", [1, 2, 3, 4])
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+@pytest.mark.parametrize("page", [0, 64])
+def test_bf16_llama_shapes(s_q, path, page):
+    d = synth.Dims(**LLAMA, s_q=s_q)
+    inp = _wl(d, 3, [s_q, 517, 1100], page=page, seed=s_q)
+    out, lse = H.run_decode(inp, path)
+    H.check_units(inp, out, lse, H.all_units(inp), "llama bf16 %s s_q=%d page=%d" % (path, s_q, page))
+
+
+@pytest.mark.parametrize("s_q", [1, 2])
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+def test_bf16_dsv3_shapes(s_q, path):
+    d = synth.Dims(**DSV3, s_q=s_q)
+    inp = _wl(d, 2, [640, 1313], page=64, seed=7)
+    out, lse = H.run_decode(inp, path)
+    H.check_units(inp, out, lse, H.sample_units(inp, 8), "dsv3 bf16 %s s_q=%d" % (path, s_q))
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 32, 128])
+@pytest.mark.parametrize("s_q", [1, 4])
+def test_bf16_group_counts(G, s_q):
+    d = synth.Dims(n_h=128, G=G, d_nope=128, d_rope=64, d_v=128, r=512, s_q=s_q)
+    inp = _wl(d, 1, [777], seed=G)
+    for path in ("absorb", "gqa"):
+        out, lse = H.run_decode(inp, path)
+        H.check_units(inp, out, lse, H.sample_units(inp, 4, seed=G), "G=%d s_q=%d %s" % (G, s_q, path))
+
+
+# ---- expansion --------------------------------------------------------------
+def test_expand_matches_oracle():
+    d = synth.Dims(**LLAMA)
+    inp = _wl(d, 2, [130, 257], page=64, seed=3)
+    kp, vp = H.run_expand(inp)
+    W_uk = inp.W_uk.double().cpu().numpy()
+    W_uv = inp.W_uv.double().cpu().numpy()
+    for b in range(2):
+        rows = inp.logical_latent(b).double().cpu().numpy()
+        L = inp.seq_lens_host[b]
+        nb = (L + 63) // 64
+        pages = inp.block_table[b, :nb].long()
+        K = kp[pages].reshape(nb * 64, d.G, d.d_qk)[:L].double().cpu().numpy()
+        V = vp[pages].reshape(nb * 64, d.G, d.d_v)[:L].double().cpu().numpy()
+        for g in range(d.G):
+            Kr, Vr = O.expand_group(rows[:, : d.r], rows[:, d.r:], W_uk[g], W_uv[g])
+            H.assert_close(K[:, g], Kr, "bf16", "K b=%d g=%d" % (b, g))
+            H.assert_close(V[:, g], Vr, "bf16", "V b=%d g=%d" % (b, g))
+            assert torch.equal(torch.tensor(K[:, g, d.d_nope:]), torch.tensor(rows[:, d.r:]))
+
+
+def test_expand_tail_only_touches_new_tokens():
+    d = synth.Dims(**LLAMA, s_q=2)
+    inp = _wl(d, 2, [300, 41], seed=5)
+    kp, vp = H.run_expand(inp)
+    sentinel = 7.0
+    kp2 = torch.full_like(kp, sentinel)
+    vp2 = torch.full_like(vp, sentinel)
+    H.run_expand(inp, tail=2, pools=(kp2, vp2))
+    for b, L in enumerate(inp.seq_lens_host):
+        assert torch.equal(kp2[b, L - 2:L], kp[b, L - 2:L])
+        assert torch.equal(vp2[b, L - 2:L], vp[b, L - 2:L])
+        assert bool((kp2[b, :L - 2] == sentinel).all()) and bool((vp2[b, L:] == sentinel).all())
+
+
+# ---- combine ------------------------------------------------------------
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_combine_matches_oracle(dtype):
+    from latent_kv_cache_flash_b200 import gqla
+    g = torch.Generator(device=DEV)
+    g.manual_seed(0)
+    S, R, D = 5, 77, 512
+    o = torch.randn((S, R, D), generator=g, device=DEV)
+    l = torch.randn((S, R), generator=g, device=DEV) * 3
+    l[1, :10] = -float("inf")
+    l[:, 20] = -float("inf")       # a row with no keys at all
+    out = torch.empty((R, D), dtype=dtype, device=DEV)
+    lse = torch.empty((R,), device=DEV)
+    gqla.gqla_splitkv_combine(o, l, out, lse)
+    ro, rl = O.splitkv_combine(o.double().cpu().numpy(), l.double().cpu().numpy())
+    H.assert_close(out.float().cpu().numpy(), ro, "f32" if dtype == torch.float32 else "bf16", "combine out")
+    H.assert_close(lse.cpu().numpy(), rl, "f32", "combine lse")
+    assert torch.all(out[20] == 0)
+
+
+# ---- invariances ------------------------------------------------------------
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+def test_paged_equals_contiguous_and_padding_poison(path):
+    d = synth.Dims(**LLAMA, s_q=2)
+    lens = [390, 1000]
+    a = _wl(d, 2, lens, page=0, seed=9)
+    # the same logical tokens in a permuted paged pool
+    b = _wl(d, 2, lens, page=64, seed=9)
+    for bb in range(2):
+        L = lens[bb]
+        nb = (L + 63) // 64
+        pages = b.block_table[bb, :nb].long()
+        pool = b.latent[pages].reshape(nb * 64, -1)
+        pool[:L] = a.latent[bb, :L]
+        pool[L:] = 1e4                       # finite poison past the end
+        b.latent[pages] = pool.reshape(nb, 64, -1)
+    b.q.copy_(a.q)
+    b.W_uk.copy_(a.W_uk)
+    b.W_uv.copy_(a.W_uv)
+    a.latent[0, lens[0]:] = -1e4
+    oa, la = H.run_decode(a, path, num_splits=3)
+    ob, lb = H.run_decode(b, path, num_splits=3)
+    assert torch.equal(oa, ob) and torch.equal(la, lb)
+
+
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+def test_split_count_invariance(path):
+    d = synth.Dims(**LLAMA)
+    inp = _wl(d, 2, [2000, 3000], seed=4)
+    ref_o, ref_l = H.run_decode(inp, path, num_splits=1)
+    for S in (2, 7, 24):
+        o, l = H.run_decode(inp, path, num_splits=S)
+        H.assert_close(o.float().cpu().numpy(), ref_o.float().cpu().numpy(), "bf16", "splits %d" % S)
+        np.testing.assert_allclose(l.cpu().numpy(), ref_l.cpu().numpy(), rtol=0, atol=2e-3)
+
+
+def test_paths_agree_full_tensor():
+    """absorb and GQA outputs of the same weights agree on the whole tensor."""
+    d = synth.Dims(**DSV3, s_q=2)
+    inp = _wl(d, 3, [700, 2048, 4000], page=64, seed=12)
+    oa, la = H.run_decode(inp, "absorb")
+    og, lg = H.run_decode(inp, "gqa")
+    H.assert_close(oa.float().cpu().numpy(), og.float().cpu().numpy(), "bf16", "absorb vs gqa")
+    np.testing.assert_allclose(la.cpu().numpy(), lg.cpu().numpy(), rtol=0, atol=2e-2)
+
+
+# ---- edge cases and device status -------------------------------------------
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+def test_edge_lengths(path):
+    d = synth.Dims(**LLAMA, s_q=3)
+    inp = _wl(d, 4, [3, 4, 129, 128], page=64, seed=2)   # L == s_q, page-boundary lengths
+    out, lse = H.run_decode(inp, path)
+    H.check_units(inp, out, lse, H.all_units(inp), "edge " + path)
+    d1 = synth.Dims(**LLAMA, s_q=1)
+    inp = _wl(d1, 1, [1], seed=2)
+    out, lse = H.run_decode(inp, path)
+    H.check_units(inp, out, lse, H.all_units(inp), "L=1 " + path)
+
+
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+def test_device_status_flags(path):
+    from latent_kv_cache_flash_b200 import gqla
+    d = synth.Dims(**LLAMA, s_q=2)
+    inp = _wl(d, 3, [100, 200, 300], page=64, seed=1)
+    pools = H.run_expand(inp) if path == "gqa" else None
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    inp.seq_lens[0] = 1                       # shorter than s_q
+    inp.block_table[2, 1] = inp.num_pages + 5  # page id outside the pool
+    out, lse = H.run_decode(inp, path, pools=pools, dev_status=st)
+    torch.cuda.synchronize()
+    flags = int(st.item())
+    assert flags & gqla.DEV_SHORT_SEQ and flags & gqla.DEV_BAD_PAGE
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
+    assert torch.all(out[2] == 0) and torch.all(torch.isneginf(lse[2]))
+    inp.seq_lens_host[0] = 1
+    inp.block_table[2, 1] = 0
+    H.check_units(inp, out, lse, [(1, g) for g in range(d.G)], "healthy row " + path)
+    st.zero_()
+    inp.seq_lens[1] = 400                     # above the host bound max_seq_len=300
+    H.run_decode(inp, path, pools=pools, dev_status=st, max_seq_len=300)
+    torch.cuda.synchronize()
+    assert int(st.item()) & gqla.DEV_OVERFLOW
+
+
+# ---- full-size workloads: whole GPU launch, sampled oracle units ------------
+@pytest.mark.parametrize("s_q", [1, 2])
+def test_llama3_8b_full_size(s_q):
+    inp = synth.make_inputs(synth.llama3_8b(s_q=s_q), DEV)
+    for path in ("absorb", "gqa"):
+        out, lse = H.run_decode(inp, path)
+        H.check_units(inp, out, lse, H.sample_units(inp, 4, seed=s_q), "llama full %s s_q=%d" % (path, s_q))
+
+
+def test_dsv3_64k_sampled():
+    inp = synth.make_inputs(synth.dsv3(seq_len=65536, s_q=2, batch=8), DEV)
+    for path in ("absorb", "gqa"):
+        out, lse = H.run_decode(inp, path)
+        H.check_units(inp, out, lse, H.sample_units(inp, 3, seed=5), "dsv3 64K %s" % path)
+
+
+def test_ragged_paged_full_size():
+    inp = synth.make_inputs(synth.ragged_paged(), DEV)
+    for path in ("absorb", "gqa"):
+        out, lse = H.run_decode(inp, path)
+        H.check_units(inp, out, lse, H.sample_units(inp, 4, seed=8), "ragged paged %s" % path)
