@@ -16,7 +16,7 @@ namespace {
 
 constexpr int kSplitGranule = 128;   // token granule of split boundaries
 constexpr int kMaxSplits = 256;
-constexpr int kMinTokensPerSplit = 256;
+constexpr int kMinTokensPerSplit = 512;
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -61,12 +61,17 @@ SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, 
   const int L = l.max_seq_len;
   int S = requested;
   if (S <= 0) {
-    // Enough CTAs for two per SM: absorb CTAs cover (sequence, 64-row head
-    // block), GQA CTAs (sequence, group).
-    long long units = path == GQLA_PATH_ABSORB
-                          ? (long long)l.batch * ((d.n_h * d.s_q + 63) / 64)
-                          : (long long)l.batch * d.G;
-    long long want = (2LL * num_sms() + units - 1) / units;
+    // Absorb CTAs cover (sequence, 64-row head block): about two per SM.
+    // GQA CTAs cover (sequence, group, 64-row block), two resident per SM:
+    // aim at six waves so the last one is nearly full.
+    long long units, want;
+    if (path == GQLA_PATH_ABSORB) {
+      units = (long long)l.batch * ((d.n_h * d.s_q + 63) / 64);
+      want = (2LL * num_sms() + units - 1) / units;
+    } else {
+      units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 63) / 64);
+      want = (12LL * num_sms() + units - 1) / units;
+    }
     long long cap = (L + kMinTokensPerSplit - 1) / kMinTokensPerSplit;
     S = (int)(want < cap ? want : cap);
   }
@@ -129,6 +134,22 @@ size_t ws_layout(const Problem& p, gqla_path path, bool tc, Workspace* ws, char*
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+cudaError_t ensure_smem_limit(const void* func, int bytes) {
+  static std::mutex mu;
+  struct Entry { const void* f; int dev; int bytes; };
+  static Entry done[256];
+  static int n_done = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> g(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].f == func && done[i].dev == dev && done[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && n_done < 256) done[n_done++] = Entry{func, dev, bytes};
+  return e;
+}
 
 int num_sms() {
   static std::mutex mu;

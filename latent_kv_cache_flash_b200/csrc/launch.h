@@ -54,4 +54,7 @@ int num_sms();
 // Counts one kernel launch (reported by gqla_launch_counter).
 void count_launch(int n = 1);
 
+// Raises a kernel's dynamic shared-memory limit once per device.
+cudaError_t ensure_smem_limit(const void* func, int bytes);
+
 }  // namespace gqla

@@ -366,11 +366,8 @@ cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, c
   prm.rows = p.rows;
   prm.st = st;
   dim3 grid(p.plan.num_splits, p.ly.batch * d.G, (rb + prm.rbc - 1) / prm.rbc);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(gqa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    attr = true;
-  }
+  cudaError_t e = ensure_smem_limit((const void*)gqa_decode_kernel, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
   gqa_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, prm);
   count_launch();
   return cudaGetLastError();
