@@ -309,7 +309,7 @@ def run_ours(args):
     launches = gqla.gqla_launch_counter() - n0
     ms_step = total_ms / args.steps
     # per-call breakdown (each over at least ~0.3 s of device time)
-    reps = max(args.steps, int(300.0 / max(ms_step, 1e-3)))
+    reps = args.steps if args.no_clocks else max(args.steps, int(300.0 / max(ms_step, 1e-3)))
     ms_absorb = timed(absorb, reps) / reps
     ms_gqa = timed(gqa, reps) / reps
     ms_tail = timed(expand_tail, reps) / reps

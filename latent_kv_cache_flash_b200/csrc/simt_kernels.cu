@@ -73,9 +73,10 @@ __global__ void expand_kernel(KvLayout ly, const T* __restrict__ latent, const T
   }
 }
 
-// q~[row, k] = sum_j W_uk[g, k, j] q_nope[row, j]  (absorbed query, fp32).
-template <typename T>
-__global__ void absorb_q_kernel(const T* __restrict__ q, const T* __restrict__ W_uk, float* __restrict__ qt,
+// q~[row, k] = sum_j W_uk[g, k, j] q_nope[row, j]  (absorbed query, fp32
+// accumulation, stored as OutT).
+template <typename T, typename OutT>
+__global__ void absorb_q_kernel(const T* __restrict__ q, const T* __restrict__ W_uk, OutT* __restrict__ qt,
                                 int n_h, int m, int d_n, int d_qk, int r) {
   extern __shared__ float sq[];  // [d_n]
   const long long row = blockIdx.x;
@@ -86,7 +87,7 @@ __global__ void absorb_q_kernel(const T* __restrict__ q, const T* __restrict__ W
     const T* w = W_uk + ((size_t)g * r + k) * d_n;
     float acc = 0.f;
     for (int j = 0; j < d_n; ++j) acc = fmaf(to_f32(w[j]), sq[j], acc);
-    qt[row * r + k] = acc;
+    qt[row * r + k] = from_f32<OutT>(acc);
   }
 }
 
@@ -244,11 +245,20 @@ cudaError_t simt_absorb_q(const Problem& p, const void* q, const void* W_uk, flo
   const auto& d = p.d;
   size_t smem = (size_t)d.d_nope * sizeof(float);
   if (d.dtype == GQLA_F32)
-    absorb_q_kernel<float><<<(unsigned)p.rows, 256, smem, s>>>((const float*)q, (const float*)W_uk, qt, d.n_h,
-                                                               p.m, d.d_nope, p.d_qk, d.r);
+    absorb_q_kernel<float, float><<<(unsigned)p.rows, 256, smem, s>>>((const float*)q, (const float*)W_uk, qt,
+                                                                      d.n_h, p.m, d.d_nope, p.d_qk, d.r);
   else
-    absorb_q_kernel<__nv_bfloat16><<<(unsigned)p.rows, 256, smem, s>>>(
+    absorb_q_kernel<__nv_bfloat16, float><<<(unsigned)p.rows, 256, smem, s>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)W_uk, qt, d.n_h, p.m, d.d_nope, p.d_qk, d.r);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t absorb_q_bf16(const Problem& p, const void* q, const void* W_uk, __nv_bfloat16* qt, cudaStream_t s) {
+  const auto& d = p.d;
+  size_t smem = (size_t)d.d_nope * sizeof(float);
+  absorb_q_kernel<__nv_bfloat16, __nv_bfloat16><<<(unsigned)p.rows, 256, smem, s>>>(
+      (const __nv_bfloat16*)q, (const __nv_bfloat16*)W_uk, qt, d.n_h, p.m, d.d_nope, p.d_qk, d.r);
   count_launch();
   return cudaGetLastError();
 }

@@ -4,11 +4,6 @@
 
 namespace gqla {
 
-bool tc_absorb_supports(const Problem&) { return false; }
-cudaError_t tc_absorb_decode(const Problem&, const void*, const void*, const void*, const void*, void*, float*,
-                             const Workspace&, int32_t*, cudaStream_t) {
-  return cudaErrorNotSupported;
-}
 bool tc_expand_supports(const Problem&) { return false; }
 cudaError_t tc_expand(const Problem&, const void*, const void*, const void*, void*, void*, int, int32_t*,
                       cudaStream_t) {
