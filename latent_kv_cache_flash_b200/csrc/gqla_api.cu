@@ -16,7 +16,6 @@ namespace {
 
 constexpr int kSplitGranule = 128;   // token granule of split boundaries
 constexpr int kMaxSplits = 256;
-constexpr int kMinTokensPerSplit = 512;
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -57,30 +56,53 @@ KvLayout to_kernel_layout(const gqla_kv_layout* l) {
 
 size_t esize(gqla_dtype t) { return t == GQLA_F32 ? 4 : 2; }
 
-SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, gqla_path path) {
-  const int L = l.max_seq_len;
-  int S = requested;
-  if (S <= 0) {
-    // Absorb CTAs cover (sequence, 64-row head block): about two per SM.
-    // GQA CTAs cover (sequence, group, 64-row block), two resident per SM:
-    // aim at six waves so the last one is nearly full.
-    long long units, want;
-    if (path == GQLA_PATH_ABSORB) {
-      units = (long long)l.batch * ((d.n_h * d.s_q + 63) / 64);
-      want = (2LL * num_sms() + units - 1) / units;
-    } else {
-      units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 63) / 64);
-      want = (12LL * num_sms() + units - 1) / units;
-    }
-    long long cap = (L + kMinTokensPerSplit - 1) / kMinTokensPerSplit;
-    S = (int)(want < cap ? want : cap);
+// Split-KV plan.  A requested count is honoured up to rounding the chunk to
+// the kernel's tile.  The automatic choice minimises a simple cost model:
+// (waves of CTAs) x (chunk tokens) x (bytes a CTA streams per token), i.e.
+// the busiest SM's traffic, plus the split partials written and read back.
+SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, gqla_path path, bool tc) {
+  const long long L = l.max_seq_len;
+  const int granule = !tc ? kSplitGranule : (path == GQLA_PATH_ABSORB ? 32 : 64);
+  auto chunk_for = [&](long long S) {
+    long long c = (L + S - 1) / S;
+    return ((c + granule - 1) / granule) * granule;
+  };
+  if (requested > 0) {
+    long long S = requested > kMaxSplits ? kMaxSplits : requested;
+    long long c = chunk_for(S);
+    return SplitPlan{(int)((L + c - 1) / c), (int)c};
   }
-  if (S < 1) S = 1;
-  if (S > kMaxSplits) S = kMaxSplits;
-  int chunk = (L + S - 1) / S;
-  chunk = ((chunk + kSplitGranule - 1) / kSplitGranule) * kSplitGranule;
-  S = (L + chunk - 1) / chunk;
-  return SplitPlan{S, chunk};
+  const long long rows = (long long)l.batch * d.s_q * d.n_h;
+  long long units, slots;
+  double unit_bytes, part_bytes;
+  if (path == GQLA_PATH_ABSORB) {
+    units = (long long)l.batch * ((d.n_h * d.s_q + 63) / 64);
+    slots = (long long)num_sms() * 1;
+    unit_bytes = 2.0 * (d.r + d.d_rope);
+    part_bytes = (double)rows * (d.r + 1) * 4 * 2;
+  } else {
+    units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 63) / 64);
+    slots = (long long)num_sms() * 2;
+    unit_bytes = 2.0 * (d.d_nope + d.d_rope + d.d_v);
+    part_bytes = (double)rows * (d.d_v + 1) * 4 * 2;
+  }
+  long long max_s = (L + granule - 1) / granule;
+  if (max_s > kMaxSplits) max_s = kMaxSplits;
+  long long best_s = 1;
+  double best = -1.0;
+  for (long long S = 1; S <= max_s; ++S) {
+    const long long c = chunk_for(S);
+    const long long Se = (L + c - 1) / c;
+    if (Se != S) continue;
+    const long long waves = (units * Se + slots - 1) / slots;
+    const double cost = (double)waves * c * unit_bytes * slots + (Se > 1 ? Se * part_bytes : 0.0);
+    if (best < 0 || cost < best * 0.999) {
+      best = cost;
+      best_s = Se;
+    }
+  }
+  const long long c = chunk_for(best_s);
+  return SplitPlan{(int)((L + c - 1) / c), (int)c};
 }
 
 gqla_status make_problem(const gqla_dims* dims, const gqla_kv_layout* layout, int num_splits, gqla_path path,
@@ -95,7 +117,9 @@ gqla_status make_problem(const gqla_dims* dims, const gqla_kv_layout* layout, in
   p->d_qk = dims->d_nope + dims->d_rope;
   p->E = dims->r + dims->d_rope;
   p->rows = (long long)layout->batch * dims->s_q * dims->n_h;
-  p->plan = make_plan(*dims, *layout, num_splits, path);
+  p->plan = SplitPlan{1, layout->max_seq_len};
+  const bool tc = path == GQLA_PATH_ABSORB ? tc_absorb_supports(*p) : tc_gqa_supports(*p);
+  p->plan = make_plan(*dims, *layout, num_splits, path, tc);
   return GQLA_OK;
 }
 
@@ -115,18 +139,19 @@ size_t ws_layout(const Problem& p, gqla_path path, bool tc, Workspace* ws, char*
   const int S = p.plan.num_splits;
   const int D = path == GQLA_PATH_ABSORB ? p.d.r : p.d.d_v;
   Workspace w{nullptr, nullptr, nullptr, nullptr};
+  auto take = [&](size_t bytes) {
+    void* ptr = base ? base + off : nullptr;
+    off = align256(off + bytes);
+    return ptr;
+  };
   if (path == GQLA_PATH_ABSORB) {
-    size_t qt_bytes = (size_t)p.rows * p.d.r * (tc ? 2 : 4);
-    w.qt = base ? base + off : nullptr;
-    off = align256(off + qt_bytes);
-    w.o_lat = base ? (float*)(base + off) : nullptr;
-    off = align256(off + (size_t)p.rows * p.d.r * 4);
+    w.qt = take((size_t)p.rows * p.d.r * (tc ? 2 : 4));
+    w.o_lat = (float*)take((size_t)p.rows * p.d.r * 4);
   }
-  if (S > 1) {
-    w.o_part = base ? (float*)(base + off) : nullptr;
-    off = align256(off + (size_t)S * p.rows * D * 4);
-    w.lse_part = base ? (float*)(base + off) : nullptr;
-    off = align256(off + (size_t)S * p.rows * 4);
+  // the tensor-core absorb kernel always writes per-split partials
+  if (S > 1 || (tc && path == GQLA_PATH_ABSORB)) {
+    w.o_part = (float*)take((size_t)S * p.rows * D * 4);
+    w.lse_part = (float*)take((size_t)S * p.rows * 4);
   }
   if (ws) *ws = w;
   return off;

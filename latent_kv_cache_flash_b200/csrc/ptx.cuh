@@ -1,6 +1,6 @@
 // Inline-PTX helpers for sm_100a: mbarriers, TMA tensor loads, ldmatrix,
 // mma.sync bf16 and the tcgen05 (TMEM) family.  Every wait on an mbarrier is
-// bounded: after kSpinLimit polls it gives up and reports false.
+// bounded in time: after about two seconds it gives up and reports false.
 #pragma once
 
 #include <cuda.h>
@@ -9,8 +9,6 @@
 
 namespace gqla {
 namespace ptx {
-
-constexpr uint32_t kSpinLimit = 1u << 26;   // polls (with backoff) before a wait gives up
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -46,13 +44,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait for the phase with the given parity to complete: polls
+// try_wait (which itself suspends the thread for a short while) and gives up
+// after about kWaitLimitNs of wall time.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (i > 64) __nanosleep(32);
+    if ((i & 1023u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
   }
-  return false;
 }
 
 // -------------------------------------------------------------------- TMA

@@ -18,7 +18,15 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
                              const void* W_uv, void* out, float* lse, const Workspace& w, int32_t* st,
                              cudaStream_t s);
 
-// Cache expansion GEMM on tcgen05.
+// Small GEMMs on mma.sync (tc_gemm.cu): absorbed queries (bf16 out), the
+// fused split combine + up-projection of the absorb path.
+bool gemm_absorb_q_supports(const Problem& p);
+cudaError_t absorb_q_mma(const Problem& p, const void* q, const void* W_uk, __nv_bfloat16* qt, cudaStream_t s);
+bool gemm_combine_up_supports(const Problem& p);
+cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const float* lse_part, const void* W_uv,
+                           void* out, float* lse_out, cudaStream_t s);
+
+// Cache expansion GEMM (tc_gemm.cu).
 bool tc_expand_supports(const Problem& p);
 cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, const void* W_uv, void* k_pool,
                       void* v_pool, int tail, int32_t* st, cudaStream_t s);

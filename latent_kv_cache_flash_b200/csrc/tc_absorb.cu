@@ -55,9 +55,8 @@ constexpr float kRescaleLog2 = 8.f;
 struct AbsorbParams {
   KvLayout ly;
   SplitPlan plan;
-  float* o_lat;    // [rows, 512] when one split
-  float* o_part;   // [S, rows, 512] when several
-  float* lse;      // final lse (one split, may be null) or lse_part
+  float* o_part;   // [S, rows, 512] normalised latent outputs of each split
+  float* lse;      // [S, rows] their log-sum-exp
   int s_q;
   int rows_unit;   // n_h * s_q rows of one sequence
   int hblocks;     // ceil(rows_unit / 64)
@@ -310,8 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float inv = empty ? 0.f : 1.f / l_tot;
     const long long grow = grow0 + row;
     float* dst = nullptr;
-    if (in_range && ok) dst = (p.o_part ? p.o_part + ((long long)split * p.rows + grow) * kR : p.o_lat + grow * kR) +
-                           half * 256;
+    if (in_range && ok) dst = p.o_part + ((long long)split * p.rows + grow) * kR + half * 256;
     for (int c = 0; c < 8; ++c) {
       uint32_t ov[32];
       if (have_o) {
@@ -328,9 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (in_range && ok && half == 0 && p.lse) {
+    if (in_range && ok && half == 0) {
       const float lse = empty ? -INFINITY : (m_tot + log2f(l_tot)) * 0.69314718055994531f;
-      p.lse[p.o_part ? (long long)split * p.rows + grow : grow] = lse;
+      p.lse[(long long)split * p.rows + grow] = lse;
     }
   }
   // ------------------------------------------------------------ teardown
@@ -390,7 +388,8 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
                              cudaStream_t s) {
   const auto& d = p.d;
   const int S = p.plan.num_splits;
-  cudaError_t e = absorb_q_bf16(p, q, W_uk, (__nv_bfloat16*)w.qt, s);
+  cudaError_t e = gemm_absorb_q_supports(p) ? absorb_q_mma(p, q, W_uk, (__nv_bfloat16*)w.qt, s)
+                                            : absorb_q_bf16(p, q, W_uk, (__nv_bfloat16*)w.qt, s);
   if (e != cudaSuccess) return e;
   long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
                                         : (long long)p.ly.num_pages * p.ly.page_size;
@@ -401,9 +400,8 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
   AbsorbParams prm;
   prm.ly = p.ly;
   prm.plan = p.plan;
-  prm.o_lat = S > 1 ? nullptr : w.o_lat;
-  prm.o_part = S > 1 ? w.o_part : nullptr;
-  prm.lse = S > 1 ? w.lse_part : lse;
+  prm.o_part = w.o_part;
+  prm.lse = w.lse_part;
   prm.s_q = d.s_q;
   prm.rows_unit = d.n_h * d.s_q;
   prm.hblocks = (prm.rows_unit + kM - 1) / kM;
@@ -417,10 +415,9 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (S > 1) {
-    e = combine(S, p.rows, kR, w.o_part, w.lse_part, w.o_lat, GQLA_F32, lse, s);
-    if (e != cudaSuccess) return e;
-  }
+  if (gemm_combine_up_supports(p)) return combine_up_mma(p, S, w.o_part, w.lse_part, W_uv, out, lse, s);
+  e = combine(S, p.rows, kR, w.o_part, w.lse_part, w.o_lat, GQLA_F32, lse, s);
+  if (e != cudaSuccess) return e;
   return simt_up_proj(p, w.o_lat, W_uv, out, s);
 }
 

@@ -1,0 +1,382 @@
+// Small bf16 GEMMs around the decode kernels, on mma.sync m16n8k16 tiles
+// (fp32 accumulate):
+//  * absorb_q:      q~[row] = W_uk^g q_nope[row]          (per group, r outputs)
+//  * combine_up:    out[row] = (LSE merge of the split partials of the latent
+//                   output)[row] W_uv^g                    (per group, d_v outputs)
+//  * expand:        K[t,g] = [c_t W_uk^g ; k_rope_t], V[t,g] = c_t W_uv^g
+//                   (the GQA path's per-group expanded cache, for all tokens
+//                   or for the newest `tail` tokens of every sequence)
+// All three read their row-major operands through ldmatrix from padded shared
+// memory; the weight operand is shared by every row of a group.
+#include <math.h>
+
+#include "ptx.cuh"
+#include "tc.h"
+
+namespace gqla {
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+__device__ __forceinline__ void ldsm_a(uint32_t base, int pitch_bytes, int row0, int k0, uint32_t* a) {
+  const int lane = threadIdx.x & 31;
+  const int row = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int col = k0 + (lane >> 4) * 8;
+  ptx::ldsm_x4(base + row * pitch_bytes + col * 2, a[0], a[1], a[2], a[3]);
+}
+// B stored [n][k] (K contiguous): fragments of n-tiles n0 and n0+8 at k-step k0.
+__device__ __forceinline__ void ldsm_b_nk(uint32_t base, int pitch_bytes, int n0, int k0, uint32_t* b) {
+  const int lane = threadIdx.x & 31;
+  const int n = n0 + (lane & 7) + (lane >> 4) * 8;
+  const int k = k0 + ((lane >> 3) & 1) * 8;
+  ptx::ldsm_x4(base + n * pitch_bytes + k * 2, b[0], b[1], b[2], b[3]);
+}
+// B stored [k][n] (N contiguous): same fragments through the transposing load.
+__device__ __forceinline__ void ldsm_b_kn(uint32_t base, int pitch_bytes, int n0, int k0, uint32_t* b) {
+  const int lane = threadIdx.x & 31;
+  const int k = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int n = n0 + (lane >> 4) * 8;
+  ptx::ldsm_x4_t(base + k * pitch_bytes + n * 2, b[0], b[1], b[2], b[3]);
+}
+
+// ------------------------------------------------------------- absorb_q
+// CTA: 64 rows of group g x 128 outputs; 4 warps of 16 rows.  K = d_nope.
+constexpr int kAqRows = 64, kAqN = 128, kAqMaxK = 256;
+
+__global__ void __launch_bounds__(128) absorb_q_mma_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_uk,
+                                                           bf16* __restrict__ qt, int rows_g, int n_h, int m,
+                                                           int d_n, int d_qk, int r) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int g = blockIdx.z, n0 = blockIdx.y * kAqN;
+  const int pitch = (d_n + 8) * 2;
+  uint8_t* sA = sm;
+  uint8_t* sB = sm + kAqRows * pitch;
+  const int gran = d_n / 8;
+  for (int i = threadIdx.x; i < kAqRows * gran; i += blockDim.x) {
+    const int rr = i / gran, c = i % gran;
+    const int lr = blockIdx.x * kAqRows + rr;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (lr < rows_g) {
+      const long long grow = (long long)(lr / m) * n_h + g * m + lr % m;
+      v = *reinterpret_cast<const uint4*>(q + grow * d_qk + c * 8);
+    }
+    *reinterpret_cast<uint4*>(sA + rr * pitch + c * 16) = v;
+  }
+  for (int i = threadIdx.x; i < kAqN * gran; i += blockDim.x) {
+    const int nn = i / gran, c = i % gran;
+    *reinterpret_cast<uint4*>(sB + nn * pitch + c * 16) =
+        *reinterpret_cast<const uint4*>(W_uk + ((size_t)g * r + n0 + nn) * d_n + c * 8);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float acc[kAqN / 8][4];
+#pragma unroll
+  for (int n = 0; n < kAqN / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
+  for (int k0 = 0; k0 < d_n; k0 += 16) {
+    uint32_t a[4];
+    ldsm_a(a_base, pitch, warp * 16, k0, a);
+#pragma unroll
+    for (int np = 0; np < kAqN / 16; ++np) {
+      uint32_t b[4];
+      ldsm_b_nk(b_base, pitch, np * 16, k0, b);
+      ptx::mma_bf16_16816(acc[2 * np], a, b[0], b[1]);
+      ptx::mma_bf16_16816(acc[2 * np + 1], a, b[2], b[3]);
+    }
+  }
+  const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const int lr = blockIdx.x * kAqRows + warp * 16 + gid + 8 * h2;
+    if (lr >= rows_g) continue;
+    const long long grow = (long long)(lr / m) * n_h + g * m + lr % m;
+#pragma unroll
+    for (int n = 0; n < kAqN / 8; ++n)
+      *reinterpret_cast<uint32_t*>(qt + grow * r + n0 + n * 8 + 2 * tig) =
+          ptx::pack_bf16(acc[n][2 * h2], acc[n][2 * h2 + 1]);
+  }
+}
+
+// ----------------------------------------------------------- combine_up
+// CTA: 16 rows of group g x d_v (128) outputs; 4 warps of 32 outputs.
+// K = r = 512 streamed through shared memory in 128-row chunks of W_uv^g.
+constexpr int kCuRows = 16, kCuK = 512, kCuN = 128, kCuKChunk = 128;
+constexpr int kCuApitch = (kCuK + 8) * 2;
+constexpr int kCuBpitch = (kCuN + 8) * 2;
+constexpr int kCuMaxS = 256;
+constexpr size_t kCuSmem = (size_t)kCuRows * kCuApitch + (size_t)kCuKChunk * kCuBpitch + kCuRows * kCuMaxS * 4;
+
+__global__ void __launch_bounds__(128) combine_up_kernel(int S, const float* __restrict__ o_part,
+                                                         const float* __restrict__ lse_part,
+                                                         const bf16* __restrict__ W_uv, bf16* __restrict__ out,
+                                                         float* __restrict__ lse_out, long long rows, int rows_g,
+                                                         int n_h, int m) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint8_t* sA = sm;
+  uint8_t* sB = sm + kCuRows * kCuApitch;
+  float* sW = reinterpret_cast<float*>(sB + kCuKChunk * kCuBpitch);   // [16][S] merge weights
+  const int g = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto grow_of = [&](int rr) -> long long {
+    const int lr = blockIdx.x * kCuRows + rr;
+    return lr < rows_g ? (long long)(lr / m) * n_h + g * m + lr % m : -1;
+  };
+  // merge weights exp(lse_s - lse) per row, and the merged lse
+  if (threadIdx.x < kCuRows) {
+    const int rr = threadIdx.x;
+    const long long grow = grow_of(rr);
+    if (grow >= 0) {
+      float mx = -INFINITY;
+      for (int s = 0; s < S; ++s) mx = fmaxf(mx, lse_part[(long long)s * rows + grow]);
+      float Z = 0.f;
+      if (mx != -INFINITY)
+        for (int s = 0; s < S; ++s) Z += expf(lse_part[(long long)s * rows + grow] - mx);
+      const float inv = mx == -INFINITY ? 0.f : 1.f / Z;
+      for (int s = 0; s < S; ++s) {
+        const float ls = lse_part[(long long)s * rows + grow];
+        sW[rr * S + s] = ls == -INFINITY ? 0.f : expf(ls - mx) * inv;
+      }
+      if (lse_out) lse_out[grow] = mx == -INFINITY ? -INFINITY : mx + logf(Z);
+    } else {
+      for (int s = 0; s < S; ++s) sW[rr * S + s] = 0.f;
+    }
+  }
+  __syncthreads();
+  // merged latent rows, rounded to bf16, as the A operand
+  for (int i = threadIdx.x; i < kCuRows * (kCuK / 4); i += blockDim.x) {
+    const int rr = i / (kCuK / 4), k4 = (i % (kCuK / 4)) * 4;
+    const long long grow = grow_of(rr);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (grow >= 0)
+      for (int s = 0; s < S; ++s) {
+        const float w = sW[rr * S + s];
+        if (w == 0.f) continue;
+        const float4 v = *reinterpret_cast<const float4*>(o_part + ((long long)s * rows + grow) * kCuK + k4);
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+      }
+    uint2 pk = make_uint2(ptx::pack_bf16(acc.x, acc.y), ptx::pack_bf16(acc.z, acc.w));
+    *reinterpret_cast<uint2*>(sA + rr * kCuApitch + k4 * 2) = pk;
+  }
+  float acc[4][4];
+#pragma unroll
+  for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
+  const bf16* Wg = W_uv + (size_t)g * kCuK * kCuN;
+  for (int kc = 0; kc < kCuK; kc += kCuKChunk) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kCuKChunk * (kCuN / 8); i += blockDim.x) {
+      const int kk = i / (kCuN / 8), c = i % (kCuN / 8);
+      *reinterpret_cast<uint4*>(sB + kk * kCuBpitch + c * 16) =
+          *reinterpret_cast<const uint4*>(Wg + (size_t)(kc + kk) * kCuN + c * 8);
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int k0 = 0; k0 < kCuKChunk; k0 += 16) {
+      uint32_t a[4];
+      ldsm_a(a_base, kCuApitch, 0, kc + k0, a);
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t b[4];
+        ldsm_b_kn(b_base, kCuBpitch, warp * 32 + np * 16, k0, b);
+        ptx::mma_bf16_16816(acc[2 * np], a, b[0], b[1]);
+        ptx::mma_bf16_16816(acc[2 * np + 1], a, b[2], b[3]);
+      }
+    }
+  }
+  const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const long long grow = grow_of(gid + 8 * h2);
+    if (grow < 0) continue;
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+      *reinterpret_cast<uint32_t*>(out + grow * kCuN + warp * 32 + n * 8 + 2 * tig) =
+          ptx::pack_bf16(acc[n][2 * h2], acc[n][2 * h2 + 1]);
+  }
+}
+
+// --------------------------------------------------------------- expand
+// CTA: 64 tokens x 256 outputs of group g (128 key-nope through W_uk^g, 128
+// values through W_uv^g); 8 warps = 4 row blocks x 2 output halves.  K = 512
+// in 64-wide chunks, double-buffered with cp.async.
+constexpr int kExR = 512, kExDn = 128, kExDv = 128, kExDr = 64, kExE = kExR + kExDr;
+constexpr int kExT = 64, kExKC = 64;
+constexpr int kExApitch = (kExKC + 8) * 2;                 // 144 B
+constexpr int kExBpitch = (kExDn + kExDv + 8) * 2;         // 528 B
+constexpr int kExAbytes = kExT * kExApitch;
+constexpr int kExBbytes = kExKC * kExBpitch;
+constexpr size_t kExSmem = 2 * (size_t)(kExAbytes + kExBbytes);
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool pred) {
+  const int sz = pred ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__global__ void __launch_bounds__(256, 2) expand_mma_kernel(KvLayout ly, const bf16* __restrict__ latent,
+                                                            const bf16* __restrict__ W_uk,
+                                                            const bf16* __restrict__ W_uv, bf16* __restrict__ kp,
+                                                            bf16* __restrict__ vp, int G, int tail, int blocks_per_seq,
+                                                            int32_t* st) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ long long srow[kExT];
+  const int g = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // which token each tile row holds (pool row, or -1)
+  if (threadIdx.x < kExT) {
+    long long row = -1;
+    int b, t;
+    if (tail > 0) {
+      const long long idx = (long long)blockIdx.x * kExT + threadIdx.x;
+      b = (int)(idx / tail);
+      t = b < ly.batch ? ly.seq_lens[b] - tail + (int)(idx % tail) : -1;
+    } else {
+      b = blockIdx.x / blocks_per_seq;
+      t = (blockIdx.x % blocks_per_seq) * kExT + threadIdx.x;
+    }
+    if (b < ly.batch) {
+      const int L = ly.seq_lens[b];
+      const bool bad = L < 1 || L > ly.max_seq_len ||
+                       (ly.page_size == 0 ? L > ly.capacity : (L + ly.page_size - 1) / ly.page_size > ly.mbps);
+      if (bad) {
+        if (g == 0 && (tail > 0 ? (int)(((long long)blockIdx.x * kExT + threadIdx.x) % tail) == 0 : t == 0))
+          flag_status(st, L < 1 ? GQLA_DEV_SHORT_SEQ : GQLA_DEV_OVERFLOW);
+      } else if (t >= 0 && t < L) {
+        row = token_row(ly, b, t, g == 0 ? st : nullptr);
+      }
+    }
+    srow[threadIdx.x] = row;
+  }
+  __syncthreads();
+  const uint32_t base = ptx::smem_u32(sm);
+  auto load_chunk = [&](int kc, int buf) {
+    const uint32_t a = base + buf * (kExAbytes + kExBbytes);
+    const uint32_t bb = a + kExAbytes;
+    for (int i = threadIdx.x; i < kExT * (kExKC / 8); i += blockDim.x) {
+      const int tt = i / (kExKC / 8), c = i % (kExKC / 8);
+      const long long row = srow[tt];
+      cp_async16(a + tt * kExApitch + c * 16, latent + (row < 0 ? 0 : row) * kExE + kc + c * 8, row >= 0);
+    }
+    for (int i = threadIdx.x; i < kExKC * ((kExDn + kExDv) / 8); i += blockDim.x) {
+      const int kk = i / ((kExDn + kExDv) / 8), c = i % ((kExDn + kExDv) / 8);
+      const bf16* src = c < kExDn / 8 ? W_uk + ((size_t)g * kExR + kc + kk) * kExDn + c * 8
+                                      : W_uv + ((size_t)g * kExR + kc + kk) * kExDv + (c - kExDn / 8) * 8;
+      cp_async16(bb + kk * kExBpitch + c * 16, src, true);
+    }
+    cp_async_commit();
+  };
+  const int wm = warp & 3, wn = warp >> 2;
+  float acc[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  load_chunk(0, 0);
+  for (int c = 0; c < kExR / kExKC; ++c) {
+    if (c + 1 < kExR / kExKC) {
+      load_chunk((c + 1) * kExKC, (c + 1) & 1);
+      cp_async_wait1();
+    } else {
+      cp_async_wait0();
+    }
+    __syncthreads();
+    const uint32_t a = base + (c & 1) * (kExAbytes + kExBbytes);
+    const uint32_t bb = a + kExAbytes;
+#pragma unroll
+    for (int k0 = 0; k0 < kExKC; k0 += 16) {
+      uint32_t af[4];
+      ldsm_a(a, kExApitch, wm * 16, k0, af);
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {
+        uint32_t b[4];
+        ldsm_b_kn(bb, kExBpitch, wn * 128 + np * 16, k0, b);
+        ptx::mma_bf16_16816(acc[2 * np], af, b[0], b[1]);
+        ptx::mma_bf16_16816(acc[2 * np + 1], af, b[2], b[3]);
+      }
+    }
+    __syncthreads();
+  }
+  const int gid = lane >> 2, tig = lane & 3;
+  constexpr int kDqk = kExDn + kExDr;
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const long long row = srow[wm * 16 + gid + 8 * h2];
+    if (row < 0) continue;
+    bf16* dst = wn == 0 ? kp + (row * G + g) * kDqk : vp + (row * G + g) * kExDv;
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+      *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * tig) = ptx::pack_bf16(acc[n][2 * h2], acc[n][2 * h2 + 1]);
+  }
+  // the shared RoPE key is copied into every group's key
+  for (int i = threadIdx.x; i < kExT * (kExDr / 8); i += blockDim.x) {
+    const int tt = i / (kExDr / 8), c = i % (kExDr / 8);
+    const long long row = srow[tt];
+    if (row < 0) continue;
+    *reinterpret_cast<uint4*>(kp + (row * G + g) * kDqk + kExDn + c * 8) =
+        *reinterpret_cast<const uint4*>(latent + row * kExE + kExR + c * 8);
+  }
+}
+
+}  // namespace
+
+bool gemm_absorb_q_supports(const Problem& p) {
+  return p.d.d_nope % 16 == 0 && p.d.d_nope <= kAqMaxK && p.d.r % kAqN == 0;
+}
+
+cudaError_t absorb_q_mma(const Problem& p, const void* q, const void* W_uk, bf16* qt, cudaStream_t s) {
+  const auto& d = p.d;
+  const int rows_g = p.ly.batch * d.s_q * p.m;
+  const int pitch = (d.d_nope + 8) * 2;
+  const size_t smem = (size_t)(kAqRows + kAqN) * pitch;
+  cudaError_t e = ensure_smem_limit((const void*)absorb_q_mma_kernel, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((rows_g + kAqRows - 1) / kAqRows, d.r / kAqN, d.G);
+  absorb_q_mma_kernel<<<grid, 128, smem, s>>>((const bf16*)q, (const bf16*)W_uk, qt, rows_g, d.n_h, p.m, d.d_nope,
+                                              p.d_qk, d.r);
+  count_launch();
+  return cudaGetLastError();
+}
+
+bool gemm_combine_up_supports(const Problem& p) {
+  return p.d.r == kCuK && p.d.d_v == kCuN && p.plan.num_splits <= kCuMaxS;
+}
+
+cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const float* lse_part, const void* W_uv,
+                           void* out, float* lse_out, cudaStream_t s) {
+  const auto& d = p.d;
+  const int rows_g = p.ly.batch * d.s_q * p.m;
+  const size_t smem = (size_t)kCuRows * kCuApitch + (size_t)kCuKChunk * kCuBpitch + (size_t)kCuRows * S * 4;
+  cudaError_t e = ensure_smem_limit((const void*)combine_up_kernel, (int)kCuSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((rows_g + kCuRows - 1) / kCuRows, d.G);
+  combine_up_kernel<<<grid, 128, smem, s>>>(S, o_part, lse_part, (const bf16*)W_uv, (bf16*)out, lse_out, p.rows,
+                                            rows_g, d.n_h, p.m);
+  count_launch();
+  return cudaGetLastError();
+}
+
+bool tc_expand_supports(const Problem& p) {
+  const auto& d = p.d;
+  return d.dtype == GQLA_BF16 && d.r == kExR && d.d_nope == kExDn && d.d_v == kExDv && d.d_rope == kExDr;
+}
+
+cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, const void* W_uv, void* k_pool,
+                      void* v_pool, int tail, int32_t* st, cudaStream_t s) {
+  const int span = tail > 0 ? (tail < p.ly.max_seq_len ? tail : p.ly.max_seq_len) : p.ly.max_seq_len;
+  const int bps = (span + kExT - 1) / kExT;
+  long long gx = tail > 0 ? ((long long)p.ly.batch * span + kExT - 1) / kExT : (long long)p.ly.batch * bps;
+  if (gx > 0x7fffffffLL) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_limit((const void*)expand_mma_kernel, (int)kExSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)gx, p.d.G);
+  expand_mma_kernel<<<grid, 256, kExSmem, s>>>(p.ly, (const bf16*)latent, (const bf16*)W_uk, (const bf16*)W_uv,
+                                               (bf16*)k_pool, (bf16*)v_pool, p.d.G, tail > 0 ? span : 0, bps, st);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace gqla
