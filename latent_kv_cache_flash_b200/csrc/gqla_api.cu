@@ -62,7 +62,7 @@ size_t esize(gqla_dtype t) { return t == GQLA_F32 ? 4 : 2; }
 // the busiest SM's traffic, plus the split partials written and read back.
 SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, gqla_path path, bool tc) {
   const long long L = l.max_seq_len;
-  const int granule = !tc ? kSplitGranule : (path == GQLA_PATH_ABSORB ? 32 : 64);
+  const int granule = !tc ? kSplitGranule : 64;
   auto chunk_for = [&](long long S) {
     long long c = (L + S - 1) / S;
     return ((c + granule - 1) / granule) * granule;

@@ -11,14 +11,14 @@
 //
 // One CTA per (key-range split, sequence, block of 64 rows):
 //  * warp 0 loads the absorbed-query tile once (64 x 576, 72 KB) and streams
-//    32-token latent tiles (36 KB) with TMA into a 4-stage mbarrier ring;
+//    64-token latent tiles (72 KB) with TMA into a 2-stage mbarrier ring;
 //  * warp 1 owns 512 TMEM columns and issues the MMAs from one thread:
-//    S = Q~ C^T as 36 tcgen05.mma (M=64, N=32, K=16) into a double-buffered
+//    S = Q~ C^T as 36 tcgen05.mma (M=64, N=64, K=16) into a double-buffered
 //    S in TMEM, and O += P C[:, :512] as 4 tcgen05.mma (M=64, N=256, K=16),
 //    reading the same latent tile as an MN-major B operand;
 //  * the M=64 accumulator uses 16 of every 32 TMEM lanes, so the two 256-wide
 //    halves of O sit interleaved at lane offsets 0 and 16 of the same 256
-//    columns; S takes columns 256..319;
+//    columns; the two S buffers take columns 256..383;
 //  * warps 2-5 read S rows from TMEM, run the online softmax in the log2
 //    domain with lazy rescaling (O is only rescaled when a row max grows by
 //    more than 2^8), write P (bf16) to shared memory, and in the end scale O
@@ -38,17 +38,17 @@ constexpr int kR = 512;
 constexpr int kDr = 64;
 constexpr int kE = kR + kDr;                 // 576 latent row elements
 constexpr int kM = 64;                       // (query, head) rows per CTA
-constexpr int kTk = 32;                      // tokens per tile
-constexpr int kStages = 4;
+constexpr int kTk = 64;                      // tokens per tile
+constexpr int kStages = 2;
 constexpr int kChunks = kE / 64;             // 128-byte column chunks of a row
 constexpr int kQChunk = kM * 128;
 constexpr int kKVChunk = kTk * 128;
 constexpr int kQBytes = kChunks * kQChunk;           // 73728
 constexpr int kStageBytes = kChunks * kKVChunk;      // 36864
-constexpr int kPBytes = kM * 128;                    // rows of 128 B (first 64 B used)
+constexpr int kPBytes = kM * 128;                    // 64 rows x 64 tokens (bf16)
 constexpr size_t kSmemBytes = (size_t)kQBytes + (size_t)kStages * kStageBytes + kPBytes + 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol = 256;
+constexpr uint32_t kSCol = 256;                  // two S buffers of kTk columns
 constexpr int kThreads = 6 * 32;
 constexpr float kRescaleLog2 = 8.f;
 
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
           if (!ok) break;
           ptx::tc_fence_after();
-          const uint32_t d = tmem + kSCol + 32u * sb;
+          const uint32_t d = tmem + kSCol + (uint32_t)kTk * sb;
           const uint32_t st_addr = kv_addr + s * kStageBytes;
 #pragma unroll
           for (int kk = 0; kk < kE / 16; ++kk) {
@@ -212,22 +212,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t0 = t_begin + j * kTk;
       if (ok) ok = ptx::mbar_wait(&s_full[sb], (j >> 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
-      uint32_t sv[32];
+      uint32_t sv[kTk];
       if (ok) {
         ptx::tc_fence_after();
-        ptx::tmem_ld32(tl + kSCol + 32u * sb, sv);
+        ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * sb, sv);
+        ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * sb + 32u, sv + 32);
         ptx::tmem_ld_wait();
       }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&s_free[sb]);
-      float pv[32];
+      float pv[kTk];
       float factor = 1.f;
       int need = 0;
       if (half == 0 && ok) {
         float mx = -INFINITY;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
+        for (int t = 0; t < kTk; ++t) {
           const float x = (t0 + t < vis) ? __uint_as_float(sv[t]) * p.scale_log2 : -INFINITY;
           pv[t] = x;
           mx = fmaxf(mx, x);
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float acc = 0.f;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
+        for (int t = 0; t < kTk; ++t) {
           const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(pv[t] - m_used);
           pv[t] = e;
           acc += e;
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_sum += acc;
       } else {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) pv[t] = 0.f;
+        for (int t = 0; t < kTk; ++t) pv[t] = 0.f;
       }
       const float f_row = __shfl_sync(0xffffffffu, factor, lane & 15);
       const bool any_rescale = __any_sync(0xffffffffu, need) != 0;
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (half == 0) {
 #pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
+        for (int g8 = 0; g8 < kTk / 8; ++g8) {
           uint4 v;
           v.x = ptx::pack_bf16(pv[8 * g8 + 0], pv[8 * g8 + 1]);
           v.y = ptx::pack_bf16(pv[8 * g8 + 2], pv[8 * g8 + 3]);
@@ -415,7 +416,8 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (gemm_combine_up_supports(p)) return combine_up_mma(p, S, w.o_part, w.lse_part, W_uv, out, lse, s);
+  if (gemm_combine_up_supports(p))
+    return combine_up_mma(p, S, w.o_part, w.lse_part, W_uv, out, lse, (__nv_bfloat16*)w.o_lat, s);
   e = combine(S, p.rows, kR, w.o_part, w.lse_part, w.o_lat, GQLA_F32, lse, s);
   if (e != cudaSuccess) return e;
   return simt_up_proj(p, w.o_lat, W_uv, out, s);

@@ -1,8 +1,8 @@
 // Small bf16 GEMMs around the decode kernels, on mma.sync m16n8k16 tiles
 // (fp32 accumulate):
 //  * absorb_q:      q~[row] = W_uk^g q_nope[row]          (per group, r outputs)
-//  * combine_up:    out[row] = (LSE merge of the split partials of the latent
-//                   output)[row] W_uv^g                    (per group, d_v outputs)
+//  * combine_lat + up_proj: LSE merge of the split partials of the latent
+//                   output (bf16), then out[row] = o_lat[row] W_uv^g
 //  * expand:        K[t,g] = [c_t W_uk^g ; k_rope_t], V[t,g] = c_t W_uv^g
 //                   (the GQA path's per-group expanded cache, for all tokens
 //                   or for the newest `tail` tokens of every sequence)
@@ -98,103 +98,145 @@ __global__ void __launch_bounds__(128) absorb_q_mma_kernel(const bf16* __restric
   }
 }
 
-// ----------------------------------------------------------- combine_up
-// CTA: 16 rows of group g x d_v (128) outputs; 4 warps of 32 outputs.
-// K = r = 512 streamed through shared memory in 128-row chunks of W_uv^g.
-constexpr int kCuRows = 16, kCuK = 512, kCuN = 128, kCuKChunk = 128;
-constexpr int kCuApitch = (kCuK + 8) * 2;
-constexpr int kCuBpitch = (kCuN + 8) * 2;
-constexpr int kCuMaxS = 256;
-constexpr size_t kCuSmem = (size_t)kCuRows * kCuApitch + (size_t)kCuKChunk * kCuBpitch + kCuRows * kCuMaxS * 4;
+// --------------------------------------------------------- combine_lat
+// LSE merge of the split partials of the absorb path's latent output, one
+// warp per (row, 128-column quarter); output rounded to bf16 for the
+// up-projection's A operand.
+constexpr int kLat = 512;
 
-__global__ void __launch_bounds__(128) combine_up_kernel(int S, const float* __restrict__ o_part,
-                                                         const float* __restrict__ lse_part,
-                                                         const bf16* __restrict__ W_uv, bf16* __restrict__ out,
-                                                         float* __restrict__ lse_out, long long rows, int rows_g,
-                                                         int n_h, int m) {
+__global__ void __launch_bounds__(256) combine_lat_kernel(int S, const float* __restrict__ o_part,
+                                                          const float* __restrict__ lse_part,
+                                                          bf16* __restrict__ o_lat, float* __restrict__ lse_out,
+                                                          long long rows) {
+  const long long wid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long row = wid >> 2;
+  const int q4 = (int)(wid & 3);
+  if (row >= rows) return;
+  float mx = -INFINITY;
+  for (int s = lane; s < S; s += 32) mx = fmaxf(mx, lse_part[(long long)s * rows + row]);
+  mx = warp_max(mx);
+  float Z = 0.f;
+  if (mx != -INFINITY)
+    for (int s = lane; s < S; s += 32) Z += expf(lse_part[(long long)s * rows + row] - mx);
+  Z = warp_sum(Z);
+  const float inv = mx == -INFINITY ? 0.f : 1.f / Z;
+  const int col = q4 * 128 + lane * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (mx != -INFINITY) {
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {
+      float4 v[4];
+      float w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float ls = lse_part[(long long)(s + u) * rows + row];
+        w[u] = ls == -INFINITY ? 0.f : expf(ls - mx) * inv;
+        v[u] = *reinterpret_cast<const float4*>(o_part + ((long long)(s + u) * rows + row) * kLat + col);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc.x = fmaf(w[u], v[u].x, acc.x);
+        acc.y = fmaf(w[u], v[u].y, acc.y);
+        acc.z = fmaf(w[u], v[u].z, acc.z);
+        acc.w = fmaf(w[u], v[u].w, acc.w);
+      }
+    }
+    for (; s < S; ++s) {
+      const float ls = lse_part[(long long)s * rows + row];
+      const float w = ls == -INFINITY ? 0.f : expf(ls - mx) * inv;
+      const float4 v = *reinterpret_cast<const float4*>(o_part + ((long long)s * rows + row) * kLat + col);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+  }
+  *reinterpret_cast<uint2*>(o_lat + row * kLat + col) =
+      make_uint2(ptx::pack_bf16(acc.x, acc.y), ptx::pack_bf16(acc.z, acc.w));
+  if (q4 == 0 && lane == 0 && lse_out) lse_out[row] = mx == -INFINITY ? -INFINITY : mx + logf(Z);
+}
+
+// ------------------------------------------------------------- up_proj
+// out[row] = o_lat[row] W_uv^g.  CTA: 64 rows of group g x 128 outputs,
+// 4 warps of 16 rows; K = 512 in 64-wide chunks, double-buffered cp.async.
+constexpr int kUpRows = 64, kUpN = 128, kUpKC = 64;
+constexpr int kUpApitch = (kUpKC + 8) * 2;     // 144 B
+constexpr int kUpBpitch = (kUpN + 8) * 2;      // 272 B
+constexpr int kUpAbytes = kUpRows * kUpApitch;
+constexpr int kUpBbytes = kUpKC * kUpBpitch;
+constexpr size_t kUpSmem = 2 * (size_t)(kUpAbytes + kUpBbytes);
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool pred) {
+  const int sz = pred ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict__ o_lat,
+                                                          const bf16* __restrict__ W_uv, bf16* __restrict__ out,
+                                                          int rows_g, int n_h, int m) {
   extern __shared__ __align__(16) uint8_t sm[];
-  uint8_t* sA = sm;
-  uint8_t* sB = sm + kCuRows * kCuApitch;
-  float* sW = reinterpret_cast<float*>(sB + kCuKChunk * kCuBpitch);   // [16][S] merge weights
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base = ptx::smem_u32(sm);
   auto grow_of = [&](int rr) -> long long {
-    const int lr = blockIdx.x * kCuRows + rr;
+    const int lr = blockIdx.x * kUpRows + rr;
     return lr < rows_g ? (long long)(lr / m) * n_h + g * m + lr % m : -1;
   };
-  // merge weights exp(lse_s - lse) per row, and the merged lse
-  if (threadIdx.x < kCuRows) {
-    const int rr = threadIdx.x;
-    const long long grow = grow_of(rr);
-    if (grow >= 0) {
-      float mx = -INFINITY;
-      for (int s = 0; s < S; ++s) mx = fmaxf(mx, lse_part[(long long)s * rows + grow]);
-      float Z = 0.f;
-      if (mx != -INFINITY)
-        for (int s = 0; s < S; ++s) Z += expf(lse_part[(long long)s * rows + grow] - mx);
-      const float inv = mx == -INFINITY ? 0.f : 1.f / Z;
-      for (int s = 0; s < S; ++s) {
-        const float ls = lse_part[(long long)s * rows + grow];
-        sW[rr * S + s] = ls == -INFINITY ? 0.f : expf(ls - mx) * inv;
-      }
-      if (lse_out) lse_out[grow] = mx == -INFINITY ? -INFINITY : mx + logf(Z);
+  const bf16* Wg = W_uv + (size_t)g * kLat * kUpN;
+  auto load_chunk = [&](int kc, int buf) {
+    const uint32_t a = base + buf * (kUpAbytes + kUpBbytes);
+    const uint32_t b = a + kUpAbytes;
+    for (int i = threadIdx.x; i < kUpRows * (kUpKC / 8); i += blockDim.x) {
+      const int rr = i / (kUpKC / 8), c = i % (kUpKC / 8);
+      const long long grow = grow_of(rr);
+      cp_async16(a + rr * kUpApitch + c * 16, o_lat + (grow < 0 ? 0 : grow) * kLat + kc + c * 8, grow >= 0);
+    }
+    for (int i = threadIdx.x; i < kUpKC * (kUpN / 8); i += blockDim.x) {
+      const int kk = i / (kUpN / 8), c = i % (kUpN / 8);
+      cp_async16(b + kk * kUpBpitch + c * 16, Wg + (size_t)(kc + kk) * kUpN + c * 8, true);
+    }
+    cp_async_commit();
+  };
+  float acc[kUpN / 8][4];
+#pragma unroll
+  for (int n = 0; n < kUpN / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  load_chunk(0, 0);
+  for (int c = 0; c < kLat / kUpKC; ++c) {
+    if (c + 1 < kLat / kUpKC) {
+      load_chunk((c + 1) * kUpKC, (c + 1) & 1);
+      cp_async_wait1();
     } else {
-      for (int s = 0; s < S; ++s) sW[rr * S + s] = 0.f;
-    }
-  }
-  __syncthreads();
-  // merged latent rows, rounded to bf16, as the A operand
-  for (int i = threadIdx.x; i < kCuRows * (kCuK / 4); i += blockDim.x) {
-    const int rr = i / (kCuK / 4), k4 = (i % (kCuK / 4)) * 4;
-    const long long grow = grow_of(rr);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (grow >= 0)
-      for (int s = 0; s < S; ++s) {
-        const float w = sW[rr * S + s];
-        if (w == 0.f) continue;
-        const float4 v = *reinterpret_cast<const float4*>(o_part + ((long long)s * rows + grow) * kCuK + k4);
-        acc.x = fmaf(w, v.x, acc.x);
-        acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z);
-        acc.w = fmaf(w, v.w, acc.w);
-      }
-    uint2 pk = make_uint2(ptx::pack_bf16(acc.x, acc.y), ptx::pack_bf16(acc.z, acc.w));
-    *reinterpret_cast<uint2*>(sA + rr * kCuApitch + k4 * 2) = pk;
-  }
-  float acc[4][4];
-#pragma unroll
-  for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-  const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
-  const bf16* Wg = W_uv + (size_t)g * kCuK * kCuN;
-  for (int kc = 0; kc < kCuK; kc += kCuKChunk) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < kCuKChunk * (kCuN / 8); i += blockDim.x) {
-      const int kk = i / (kCuN / 8), c = i % (kCuN / 8);
-      *reinterpret_cast<uint4*>(sB + kk * kCuBpitch + c * 16) =
-          *reinterpret_cast<const uint4*>(Wg + (size_t)(kc + kk) * kCuN + c * 8);
+      cp_async_wait0();
     }
     __syncthreads();
-#pragma unroll 4
-    for (int k0 = 0; k0 < kCuKChunk; k0 += 16) {
-      uint32_t a[4];
-      ldsm_a(a_base, kCuApitch, 0, kc + k0, a);
+    const uint32_t a = base + (c & 1) * (kUpAbytes + kUpBbytes);
+    const uint32_t b = a + kUpAbytes;
 #pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        uint32_t b[4];
-        ldsm_b_kn(b_base, kCuBpitch, warp * 32 + np * 16, k0, b);
-        ptx::mma_bf16_16816(acc[2 * np], a, b[0], b[1]);
-        ptx::mma_bf16_16816(acc[2 * np + 1], a, b[2], b[3]);
+    for (int k0 = 0; k0 < kUpKC; k0 += 16) {
+      uint32_t af[4];
+      ldsm_a(a, kUpApitch, warp * 16, k0, af);
+#pragma unroll
+      for (int np = 0; np < kUpN / 16; ++np) {
+        uint32_t bf[4];
+        ldsm_b_kn(b, kUpBpitch, np * 16, k0, bf);
+        ptx::mma_bf16_16816(acc[2 * np], af, bf[0], bf[1]);
+        ptx::mma_bf16_16816(acc[2 * np + 1], af, bf[2], bf[3]);
       }
     }
+    __syncthreads();
   }
   const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
-    const long long grow = grow_of(gid + 8 * h2);
+    const long long grow = grow_of(warp * 16 + gid + 8 * h2);
     if (grow < 0) continue;
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
-      *reinterpret_cast<uint32_t*>(out + grow * kCuN + warp * 32 + n * 8 + 2 * tig) =
+    for (int n = 0; n < kUpN / 8; ++n)
+      *reinterpret_cast<uint32_t*>(out + grow * kUpN + n * 8 + 2 * tig) =
           ptx::pack_bf16(acc[n][2 * h2], acc[n][2 * h2 + 1]);
   }
 }
@@ -210,14 +252,6 @@ constexpr int kExBpitch = (kExDn + kExDv + 8) * 2;         // 528 B
 constexpr int kExAbytes = kExT * kExApitch;
 constexpr int kExBbytes = kExKC * kExBpitch;
 constexpr size_t kExSmem = 2 * (size_t)(kExAbytes + kExBbytes);
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool pred) {
-  const int sz = pred ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __global__ void __launch_bounds__(256, 2) expand_mma_kernel(KvLayout ly, const bf16* __restrict__ latent,
                                                             const bf16* __restrict__ W_uk,
@@ -342,19 +376,22 @@ cudaError_t absorb_q_mma(const Problem& p, const void* q, const void* W_uk, bf16
 }
 
 bool gemm_combine_up_supports(const Problem& p) {
-  return p.d.r == kCuK && p.d.d_v == kCuN && p.plan.num_splits <= kCuMaxS;
+  return p.d.r == kLat && p.d.d_v == kUpN;
 }
 
 cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const float* lse_part, const void* W_uv,
-                           void* out, float* lse_out, cudaStream_t s) {
+                           void* out, float* lse_out, bf16* o_lat, cudaStream_t s) {
   const auto& d = p.d;
-  const int rows_g = p.ly.batch * d.s_q * p.m;
-  const size_t smem = (size_t)kCuRows * kCuApitch + (size_t)kCuKChunk * kCuBpitch + (size_t)kCuRows * S * 4;
-  cudaError_t e = ensure_smem_limit((const void*)combine_up_kernel, (int)kCuSmem);
+  const long long warps = p.rows * 4;
+  combine_lat_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(S, o_part, lse_part, o_lat, lse_out, p.rows);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 grid((rows_g + kCuRows - 1) / kCuRows, d.G);
-  combine_up_kernel<<<grid, 128, smem, s>>>(S, o_part, lse_part, (const bf16*)W_uv, (bf16*)out, lse_out, p.rows,
-                                            rows_g, d.n_h, p.m);
+  const int rows_g = p.ly.batch * d.s_q * p.m;
+  e = ensure_smem_limit((const void*)up_proj_mma_kernel, (int)kUpSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((rows_g + kUpRows - 1) / kUpRows, d.G);
+  up_proj_mma_kernel<<<grid, 128, kUpSmem, s>>>(o_lat, (const bf16*)W_uv, (bf16*)out, rows_g, d.n_h, p.m);
   count_launch();
   return cudaGetLastError();
 }
