@@ -12,10 +12,11 @@
 // One CTA per (key-range split, sequence, block of 64 rows):
 //  * warp 0 loads the absorbed-query tile once (64 x 576, 72 KB) and streams
 //    64-token latent tiles (72 KB) with TMA into a 2-stage mbarrier ring;
-//  * warp 1 owns 512 TMEM columns and issues the MMAs from one thread:
-//    S = Q~ C^T as 36 tcgen05.mma (M=64, N=64, K=16) into a double-buffered
-//    S in TMEM, and O += P C[:, :512] as 4 tcgen05.mma (M=64, N=256, K=16),
-//    reading the same latent tile as an MN-major B operand;
+//  * warp 1 owns 512 TMEM columns and issues S = Q~ C^T as 36 tcgen05.mma
+//    (M=64, N=64, K=16) into a double-buffered S in TMEM; warp 6 issues
+//    O += P C[:, :512] as 8 tcgen05.mma (M=64, N=256, K=16), reading the same
+//    latent tile as an MN-major B operand.  Two issuing threads keep the
+//    stage release (after PV) independent of the next tile's QK issue;
 //  * the M=64 accumulator uses 16 of every 32 TMEM lanes, so the two 256-wide
 //    halves of O sit interleaved at lane offsets 0 and 16 of the same 256
 //    columns; the two S buffers take columns 256..383;
@@ -49,7 +50,7 @@ constexpr int kPBytes = kM * 128;                    // 64 rows x 64 tokens (bf1
 constexpr size_t kSmemBytes = (size_t)kQBytes + (size_t)kStages * kStageBytes + kPBytes + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 256;                  // two S buffers of kTk columns
-constexpr int kThreads = 6 * 32;
+constexpr int kThreads = 7 * 32;
 constexpr float kRescaleLog2 = 8.f;
 
 struct AbsorbParams {
@@ -73,7 +74,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + kQBytes;
   uint8_t* sP = sKV + kStages * kStageBytes;
-  __shared__ __align__(8) uint64_t q_full, p_full, pv_done, mma_drain;
+  __shared__ __align__(8) uint64_t q_full, p_full, pv_done, qk_drain, pv_drain;
   __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -86,7 +87,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(&q_full, 1);
     ptx::mbar_init(&p_full, 4);
     ptx::mbar_init(&pv_done, 1);
-    ptx::mbar_init(&mma_drain, 1);
+    ptx::mbar_init(&qk_drain, 1);
+    ptx::mbar_init(&pv_drain, 1);
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(&kv_full[s], 1);
       ptx::mbar_init(&kv_empty[s], 1);
@@ -142,56 +144,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
+    // ---------------------------------------------- QK issuer, TMEM owner
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = ptx::idesc_bf16(kM, kTk, false, false);
-      constexpr uint32_t idesc_pv = ptx::idesc_bf16(kM, 256, false, true);
-      const uint32_t q_addr = ptx::smem_u32(sQ), kv_addr = ptx::smem_u32(sKV), p_addr = ptx::smem_u32(sP);
+      const uint32_t q_addr = ptx::smem_u32(sQ), kv_addr = ptx::smem_u32(sKV);
       bool ok = ptx::mbar_wait(&q_full, 0);
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          const int s = j % kStages, sb = j & 1;
-          ok = ptx::mbar_wait(&kv_full[s], (j / kStages) & 1);
-          if (ok && j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const uint32_t d = tmem + kSCol + (uint32_t)kTk * sb;
-          const uint32_t st_addr = kv_addr + s * kStageBytes;
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kStages, sb = j & 1;
+        ok = ptx::mbar_wait(&kv_full[s], (j / kStages) & 1);
+        if (ok && j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint32_t d = tmem + kSCol + (uint32_t)kTk * sb;
+        const uint32_t st_addr = kv_addr + s * kStageBytes;
 #pragma unroll
-          for (int kk = 0; kk < kE / 16; ++kk) {
-            const uint32_t koff = (kk >> 2), kin = (kk & 3) * 32;
-            const uint64_t a = ptx::umma_desc_sw128(q_addr + koff * kQChunk + kin, 16, 1024);
-            const uint64_t bd = ptx::umma_desc_sw128(st_addr + koff * kKVChunk + kin, 16, 1024);
-            ptx::umma_bf16(d, a, bd, idesc_qk, kk > 0);
-          }
-          ptx::umma_commit(&s_full[sb]);
+        for (int kk = 0; kk < kE / 16; ++kk) {
+          const uint32_t koff = (kk >> 2), kin = (kk & 3) * 32;
+          const uint64_t a = ptx::umma_desc_sw128(q_addr + koff * kQChunk + kin, 16, 1024);
+          const uint64_t bd = ptx::umma_desc_sw128(st_addr + koff * kKVChunk + kin, 16, 1024);
+          ptx::umma_bf16(d, a, bd, idesc_qk, kk > 0);
         }
-        if (j >= 1) {
-          const int jj = j - 1, s2 = jj % kStages;
-          ok = ptx::mbar_wait(&p_full, jj & 1);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const uint32_t st_addr = kv_addr + s2 * kStageBytes;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int kk = 0; kk < kTk / 16; ++kk) {
-              const uint64_t a = ptx::umma_desc_sw128(p_addr + kk * 32, 16, 1024);
-              const uint64_t bd = ptx::umma_desc_sw128(st_addr + (4 * h) * kKVChunk + kk * 16 * 128, kKVChunk, 1024);
-              ptx::umma_bf16(tmem + (h ? (16u << 16) : 0u), a, bd, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-            }
-          }
-          ptx::umma_commit(&pv_done);
-          ptx::umma_commit(&kv_empty[s2]);
-        }
+        ptx::umma_commit(&s_full[sb]);
       }
       if (!ok) {
         flag_status(p.st, GQLA_DEV_TIMEOUT);
         atomicExch(&abort_flag, 1);
       }
       // every issued MMA has finished before TMEM is released
-      ptx::umma_commit(&mma_drain);
-      ptx::mbar_wait(&mma_drain, 0);
+      ptx::umma_commit(&qk_drain);
+      ptx::mbar_wait(&qk_drain, 0);
+    }
+  } else if (warp == 6) {
+    // ---------------------------------------------------------- PV issuer
+    // A second issuing thread: PV(j) goes out as soon as P(j) is ready, so
+    // the stage it releases is not held behind the next tile's QK.
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t idesc_pv = ptx::idesc_bf16(kM, 256, false, true);
+      const uint32_t kv_addr = ptx::smem_u32(sKV), p_addr = ptx::smem_u32(sP);
+      bool ok = true;
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kStages;
+        ok = ptx::mbar_wait(&p_full, j & 1);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint32_t st_addr = kv_addr + s * kStageBytes;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int kk = 0; kk < kTk / 16; ++kk) {
+            const uint64_t a = ptx::umma_desc_sw128(p_addr + kk * 32, 16, 1024);
+            const uint64_t bd = ptx::umma_desc_sw128(st_addr + (4 * h) * kKVChunk + kk * 16 * 128, kKVChunk, 1024);
+            ptx::umma_bf16(tmem + (h ? (16u << 16) : 0u), a, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        ptx::umma_commit(&pv_done);
+        ptx::umma_commit(&kv_empty[s]);
+      }
+      if (!ok) {
+        flag_status(p.st, GQLA_DEV_TIMEOUT);
+        atomicExch(&abort_flag, 1);
+      }
+      ptx::umma_commit(&pv_drain);
+      ptx::mbar_wait(&pv_drain, 0);
     }
   } else {
     // ------------------------------------------- softmax + epilogue warps
