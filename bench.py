@@ -50,6 +50,7 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
     return ap.parse_args()
 
 
@@ -305,9 +306,20 @@ def run_ours(args):
         clocks.start()
         time.sleep(0.3)
     n0 = gqla.gqla_launch_counter()
-    total_ms = timed(step, args.steps)
+    eager_ms = timed(step, args.steps) / args.steps
     launches = gqla.gqla_launch_counter() - n0
-    ms_step = total_ms / args.steps
+    # the same step captured once as a CUDA graph and replayed (no host
+    # launch gaps between the kernels); every kernel still runs each step
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        ms_step = timed(graph.replay, args.steps) / args.steps
+    else:
+        ms_step = eager_ms
     # per-call breakdown (each over at least ~0.3 s of device time)
     reps = args.steps if args.no_clocks else max(args.steps, int(300.0 / max(ms_step, 1e-3)))
     ms_absorb = timed(absorb, reps) / reps
@@ -382,6 +394,8 @@ def run_ours(args):
                    "seq_len": wl.seq_len, "s_q": d.s_q, "n_h": d.n_h, "G": d.G, "d_nope": d.d_nope,
                    "d_rope": d.d_rope, "d_v": d.d_v, "r": d.r,
                    "step": "expand s_q new tokens + absorb decode + GQA decode",
+                   "launch": "cuda_graph replay of the step" if graph is not None else "eager",
+                   "eager_ms_per_step": eager_ms,
                    "l2": "no flush: inputs larger than L2 (latent %.0f MB, expanded cache %.0f MB)" % (
                        alg["absorb_bytes"] / 1e6, alg["gqa_bytes"] / 1e6),
                    "parallelism": "replicas x%d (batch-sharded, no collective)" % world},
@@ -404,6 +418,7 @@ def run_ours(args):
         line["cpu_baseline"] = cpu_baseline(inp_cpu)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -41,8 +41,9 @@ __device__ __forceinline__ void ldsm_b_kn(uint32_t base, int pitch_bytes, int n0
 }
 
 // ------------------------------------------------------------- absorb_q
-// CTA: 64 rows of group g x 128 outputs; 4 warps of 16 rows.  K = d_nope.
-constexpr int kAqRows = 64, kAqN = 128, kAqMaxK = 256;
+// CTA: 32 rows of group g x 128 outputs; 4 warps = 2 row blocks x 2 output
+// halves.  K = d_nope.
+constexpr int kAqRows = 32, kAqN = 128, kAqMaxK = 256;
 
 __global__ void __launch_bounds__(128) absorb_q_mma_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_uk,
                                                            bf16* __restrict__ qt, int rows_g, int n_h, int m,
@@ -70,17 +71,18 @@ __global__ void __launch_bounds__(128) absorb_q_mma_kernel(const bf16* __restric
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float acc[kAqN / 8][4];
+  const int wr = warp & 1, wn = warp >> 1;
+  float acc[kAqN / 16][4];
 #pragma unroll
-  for (int n = 0; n < kAqN / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  for (int n = 0; n < kAqN / 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
   const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
   for (int k0 = 0; k0 < d_n; k0 += 16) {
     uint32_t a[4];
-    ldsm_a(a_base, pitch, warp * 16, k0, a);
+    ldsm_a(a_base, pitch, wr * 16, k0, a);
 #pragma unroll
-    for (int np = 0; np < kAqN / 16; ++np) {
+    for (int np = 0; np < kAqN / 32; ++np) {
       uint32_t b[4];
-      ldsm_b_nk(b_base, pitch, np * 16, k0, b);
+      ldsm_b_nk(b_base, pitch, wn * (kAqN / 2) + np * 16, k0, b);
       ptx::mma_bf16_16816(acc[2 * np], a, b[0], b[1]);
       ptx::mma_bf16_16816(acc[2 * np + 1], a, b[2], b[3]);
     }
@@ -88,12 +90,12 @@ __global__ void __launch_bounds__(128) absorb_q_mma_kernel(const bf16* __restric
   const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
-    const int lr = blockIdx.x * kAqRows + warp * 16 + gid + 8 * h2;
+    const int lr = blockIdx.x * kAqRows + wr * 16 + gid + 8 * h2;
     if (lr >= rows_g) continue;
     const long long grow = (long long)(lr / m) * n_h + g * m + lr % m;
 #pragma unroll
-    for (int n = 0; n < kAqN / 8; ++n)
-      *reinterpret_cast<uint32_t*>(qt + grow * r + n0 + n * 8 + 2 * tig) =
+    for (int n = 0; n < kAqN / 16; ++n)
+      *reinterpret_cast<uint32_t*>(qt + grow * r + n0 + wn * (kAqN / 2) + n * 8 + 2 * tig) =
           ptx::pack_bf16(acc[n][2 * h2], acc[n][2 * h2 + 1]);
   }
 }
@@ -158,9 +160,9 @@ __global__ void __launch_bounds__(256) combine_lat_kernel(int S, const float* __
 }
 
 // ------------------------------------------------------------- up_proj
-// out[row] = o_lat[row] W_uv^g.  CTA: 64 rows of group g x 128 outputs,
-// 4 warps of 16 rows; K = 512 in 64-wide chunks, double-buffered cp.async.
-constexpr int kUpRows = 64, kUpN = 128, kUpKC = 64;
+// out[row] = o_lat[row] W_uv^g.  CTA: 16 rows of group g x 128 outputs,
+// 4 warps of 32 outputs; K = 512 in 64-wide chunks, double-buffered cp.async.
+constexpr int kUpRows = 16, kUpN = 128, kUpKC = 64;
 constexpr int kUpApitch = (kUpKC + 8) * 2;     // 144 B
 constexpr int kUpBpitch = (kUpN + 8) * 2;      // 272 B
 constexpr int kUpAbytes = kUpRows * kUpApitch;
@@ -201,9 +203,9 @@ __global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict
     }
     cp_async_commit();
   };
-  float acc[kUpN / 8][4];
+  float acc[4][4];
 #pragma unroll
-  for (int n = 0; n < kUpN / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
   load_chunk(0, 0);
   for (int c = 0; c < kLat / kUpKC; ++c) {
     if (c + 1 < kLat / kUpKC) {
@@ -218,11 +220,11 @@ __global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict
 #pragma unroll
     for (int k0 = 0; k0 < kUpKC; k0 += 16) {
       uint32_t af[4];
-      ldsm_a(a, kUpApitch, warp * 16, k0, af);
+      ldsm_a(a, kUpApitch, 0, k0, af);
 #pragma unroll
-      for (int np = 0; np < kUpN / 16; ++np) {
+      for (int np = 0; np < 2; ++np) {
         uint32_t bf[4];
-        ldsm_b_kn(b, kUpBpitch, np * 16, k0, bf);
+        ldsm_b_kn(b, kUpBpitch, warp * 32 + np * 16, k0, bf);
         ptx::mma_bf16_16816(acc[2 * np], af, bf[0], bf[1]);
         ptx::mma_bf16_16816(acc[2 * np + 1], af, bf[2], bf[3]);
       }
@@ -232,35 +234,36 @@ __global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict
   const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
-    const long long grow = grow_of(warp * 16 + gid + 8 * h2);
+    const long long grow = grow_of(gid + 8 * h2);
     if (grow < 0) continue;
 #pragma unroll
-    for (int n = 0; n < kUpN / 8; ++n)
-      *reinterpret_cast<uint32_t*>(out + grow * kUpN + n * 8 + 2 * tig) =
+    for (int n = 0; n < 4; ++n)
+      *reinterpret_cast<uint32_t*>(out + grow * kUpN + warp * 32 + n * 8 + 2 * tig) =
           ptx::pack_bf16(acc[n][2 * h2], acc[n][2 * h2 + 1]);
   }
 }
 
 // --------------------------------------------------------------- expand
-// CTA: 64 tokens x 256 outputs of group g (128 key-nope through W_uk^g, 128
-// values through W_uv^g); 8 warps = 4 row blocks x 2 output halves.  K = 512
-// in 64-wide chunks, double-buffered with cp.async.
+// CTA: 64 tokens x 64 outputs of group g (quarter q of its 256 outputs: q = 0,1
+// key-nope through W_uk^g, q = 2,3 values through W_uv^g); 4 warps of 16 rows.
+// K = 512 in 64-wide chunks, double-buffered with cp.async.  Quarter 0 also
+// copies the shared RoPE key into the group's key.
 constexpr int kExR = 512, kExDn = 128, kExDv = 128, kExDr = 64, kExE = kExR + kExDr;
-constexpr int kExT = 64, kExKC = 64;
+constexpr int kExT = 64, kExKC = 64, kExN = 64;
 constexpr int kExApitch = (kExKC + 8) * 2;                 // 144 B
-constexpr int kExBpitch = (kExDn + kExDv + 8) * 2;         // 528 B
+constexpr int kExBpitch = (kExN + 8) * 2;                  // 144 B
 constexpr int kExAbytes = kExT * kExApitch;
 constexpr int kExBbytes = kExKC * kExBpitch;
 constexpr size_t kExSmem = 2 * (size_t)(kExAbytes + kExBbytes);
 
-__global__ void __launch_bounds__(256, 2) expand_mma_kernel(KvLayout ly, const bf16* __restrict__ latent,
-                                                            const bf16* __restrict__ W_uk,
-                                                            const bf16* __restrict__ W_uv, bf16* __restrict__ kp,
-                                                            bf16* __restrict__ vp, int G, int tail, int blocks_per_seq,
-                                                            int32_t* st) {
+__global__ void __launch_bounds__(128) expand_mma_kernel(KvLayout ly, const bf16* __restrict__ latent,
+                                                         const bf16* __restrict__ W_uk,
+                                                         const bf16* __restrict__ W_uv, bf16* __restrict__ kp,
+                                                         bf16* __restrict__ vp, int G, int tail, int blocks_per_seq,
+                                                         int32_t* st) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ long long srow[kExT];
-  const int g = blockIdx.y;
+  const int g = blockIdx.y, quarter = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // which token each tile row holds (pool row, or -1)
   if (threadIdx.x < kExT) {
@@ -278,16 +281,21 @@ __global__ void __launch_bounds__(256, 2) expand_mma_kernel(KvLayout ly, const b
       const int L = ly.seq_lens[b];
       const bool bad = L < 1 || L > ly.max_seq_len ||
                        (ly.page_size == 0 ? L > ly.capacity : (L + ly.page_size - 1) / ly.page_size > ly.mbps);
+      const bool reporter = g == 0 && quarter == 0 &&
+                            (tail > 0 ? (int)(((long long)blockIdx.x * kExT + threadIdx.x) % tail) == 0 : t == 0);
       if (bad) {
-        if (g == 0 && (tail > 0 ? (int)(((long long)blockIdx.x * kExT + threadIdx.x) % tail) == 0 : t == 0))
-          flag_status(st, L < 1 ? GQLA_DEV_SHORT_SEQ : GQLA_DEV_OVERFLOW);
+        if (reporter) flag_status(st, L < 1 ? GQLA_DEV_SHORT_SEQ : GQLA_DEV_OVERFLOW);
       } else if (t >= 0 && t < L) {
-        row = token_row(ly, b, t, g == 0 ? st : nullptr);
+        row = token_row(ly, b, t, (g == 0 && quarter == 0) ? st : nullptr);
       }
     }
     srow[threadIdx.x] = row;
   }
   __syncthreads();
+  const bool is_k = quarter < 2;
+  const bf16* Wsrc = is_k ? W_uk + (size_t)g * kExR * kExDn + quarter * kExN
+                          : W_uv + (size_t)g * kExR * kExDv + (quarter - 2) * kExN;
+  const int wld = is_k ? kExDn : kExDv;
   const uint32_t base = ptx::smem_u32(sm);
   auto load_chunk = [&](int kc, int buf) {
     const uint32_t a = base + buf * (kExAbytes + kExBbytes);
@@ -297,18 +305,15 @@ __global__ void __launch_bounds__(256, 2) expand_mma_kernel(KvLayout ly, const b
       const long long row = srow[tt];
       cp_async16(a + tt * kExApitch + c * 16, latent + (row < 0 ? 0 : row) * kExE + kc + c * 8, row >= 0);
     }
-    for (int i = threadIdx.x; i < kExKC * ((kExDn + kExDv) / 8); i += blockDim.x) {
-      const int kk = i / ((kExDn + kExDv) / 8), c = i % ((kExDn + kExDv) / 8);
-      const bf16* src = c < kExDn / 8 ? W_uk + ((size_t)g * kExR + kc + kk) * kExDn + c * 8
-                                      : W_uv + ((size_t)g * kExR + kc + kk) * kExDv + (c - kExDn / 8) * 8;
-      cp_async16(bb + kk * kExBpitch + c * 16, src, true);
+    for (int i = threadIdx.x; i < kExKC * (kExN / 8); i += blockDim.x) {
+      const int kk = i / (kExN / 8), c = i % (kExN / 8);
+      cp_async16(bb + kk * kExBpitch + c * 16, Wsrc + (size_t)(kc + kk) * wld + c * 8, true);
     }
     cp_async_commit();
   };
-  const int wm = warp & 3, wn = warp >> 2;
-  float acc[16][4];
+  float acc[kExN / 8][4];
 #pragma unroll
-  for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  for (int n = 0; n < kExN / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
   load_chunk(0, 0);
   for (int c = 0; c < kExR / kExKC; ++c) {
     if (c + 1 < kExR / kExKC) {
@@ -323,11 +328,11 @@ __global__ void __launch_bounds__(256, 2) expand_mma_kernel(KvLayout ly, const b
 #pragma unroll
     for (int k0 = 0; k0 < kExKC; k0 += 16) {
       uint32_t af[4];
-      ldsm_a(a, kExApitch, wm * 16, k0, af);
+      ldsm_a(a, kExApitch, warp * 16, k0, af);
 #pragma unroll
-      for (int np = 0; np < 8; ++np) {
+      for (int np = 0; np < kExN / 16; ++np) {
         uint32_t b[4];
-        ldsm_b_kn(bb, kExBpitch, wn * 128 + np * 16, k0, b);
+        ldsm_b_kn(bb, kExBpitch, np * 16, k0, b);
         ptx::mma_bf16_16816(acc[2 * np], af, b[0], b[1]);
         ptx::mma_bf16_16816(acc[2 * np + 1], af, b[2], b[3]);
       }
@@ -338,20 +343,22 @@ __global__ void __launch_bounds__(256, 2) expand_mma_kernel(KvLayout ly, const b
   constexpr int kDqk = kExDn + kExDr;
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
-    const long long row = srow[wm * 16 + gid + 8 * h2];
+    const long long row = srow[warp * 16 + gid + 8 * h2];
     if (row < 0) continue;
-    bf16* dst = wn == 0 ? kp + (row * G + g) * kDqk : vp + (row * G + g) * kExDv;
+    bf16* dst = is_k ? kp + (row * G + g) * kDqk + quarter * kExN : vp + (row * G + g) * kExDv + (quarter - 2) * kExN;
 #pragma unroll
-    for (int n = 0; n < 16; ++n)
+    for (int n = 0; n < kExN / 8; ++n)
       *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * tig) = ptx::pack_bf16(acc[n][2 * h2], acc[n][2 * h2 + 1]);
   }
-  // the shared RoPE key is copied into every group's key
-  for (int i = threadIdx.x; i < kExT * (kExDr / 8); i += blockDim.x) {
-    const int tt = i / (kExDr / 8), c = i % (kExDr / 8);
-    const long long row = srow[tt];
-    if (row < 0) continue;
-    *reinterpret_cast<uint4*>(kp + (row * G + g) * kDqk + kExDn + c * 8) =
-        *reinterpret_cast<const uint4*>(latent + row * kExE + kExR + c * 8);
+  if (quarter == 0) {
+    // the shared RoPE key is copied into every group's key
+    for (int i = threadIdx.x; i < kExT * (kExDr / 8); i += blockDim.x) {
+      const int tt = i / (kExDr / 8), c = i % (kExDr / 8);
+      const long long row = srow[tt];
+      if (row < 0) continue;
+      *reinterpret_cast<uint4*>(kp + (row * G + g) * kDqk + kExDn + c * 8) =
+          *reinterpret_cast<const uint4*>(latent + row * kExE + kExR + c * 8);
+    }
   }
 }
 
@@ -409,8 +416,8 @@ cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, co
   if (gx > 0x7fffffffLL) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_limit((const void*)expand_mma_kernel, (int)kExSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)gx, p.d.G);
-  expand_mma_kernel<<<grid, 256, kExSmem, s>>>(p.ly, (const bf16*)latent, (const bf16*)W_uk, (const bf16*)W_uv,
+  dim3 grid((unsigned)gx, p.d.G, 4);
+  expand_mma_kernel<<<grid, 128, kExSmem, s>>>(p.ly, (const bf16*)latent, (const bf16*)W_uk, (const bf16*)W_uv,
                                                (bf16*)k_pool, (bf16*)v_pool, p.d.G, tail > 0 ? span : 0, bps, st);
   count_launch();
   return cudaGetLastError();
