@@ -159,6 +159,26 @@ gqla_status gqla_decode_gqa(const gqla_dims* dims, const gqla_kv_layout* layout,
                             void* workspace, size_t workspace_bytes,
                             int32_t* dev_status, void* stream);
 
+/* gqla_decode_gqa without a workspace argument, for callers that cannot
+ * allocate device memory: a plug-in whose host framework owns every byte of
+ * device memory and gives it no allocator, or a decode loop that must not call
+ * cudaMalloc/cudaFree (they synchronise the device) on its hot path.  The
+ * pages have no counterpart to this call; it is a deployment convenience.
+ *   Same arguments, layouts, results and errors as gqla_decode_gqa, minus the
+ *   workspace.  The split scratch is a library-owned device array of 32 MiB,
+ *   reserved on every GPU that loads the library and held until the process
+ *   exits.  A problem whose split scratch would exceed 32 MiB (about
+ *   num_splits * B * s_q * n_h * (d_v + 1) * 4 bytes) is refused with
+ *   GQLA_ERR_WORKSPACE before any launch: pass a smaller num_splits.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one array, so calls whose kernels may overlap on the
+ *   GPU (different streams, or other threads) race: serialise them. */
+gqla_status gqla_decode_gqa_noalloc(const gqla_dims* dims, const gqla_kv_layout* layout,
+                                    const void* q, const void* k_pool, const void* v_pool,
+                                    void* out, float* lse, int32_t num_splits,
+                                    int32_t* dev_status, void* stream);
+
 /* Log-sum-exp merge of attention results over disjoint key ranges:
  *   lse[row] = ln sum_j exp(lse_part[j,row]);
  *   out[row] = sum_j exp(lse_part[j,row] - lse[row]) * o_part[j,row,:]

@@ -105,6 +105,8 @@ SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, 
   return SplitPlan{(int)((L + c - 1) / c), (int)c};
 }
 
+}  // namespace
+
 gqla_status make_problem(const gqla_dims* dims, const gqla_kv_layout* layout, int num_splits, gqla_path path,
                          Problem* p) {
   gqla_status s = check_dims(dims);
@@ -131,8 +133,6 @@ bool simt_supports(const Problem& p, gqla_path path) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-}  // namespace
 
 size_t ws_layout(const Problem& p, gqla_path path, bool tc, Workspace* ws, char* base) {
   size_t off = 0;

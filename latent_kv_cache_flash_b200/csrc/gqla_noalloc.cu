@@ -1,0 +1,85 @@
+// gqla_decode_gqa_noalloc: the GQA decode entry point without a caller-supplied
+// workspace.  Its split-KV scratch (per-split partial outputs and their
+// log-sum-exp) lives in one file-scope device array of fixed size, so the call
+// needs no allocation at all: for hosts that own every byte of device memory
+// and hand a plug-in none of it, and for decode loops that may not call an
+// allocator on the hot path (cudaMalloc/cudaFree synchronise the device).
+#include <mutex>
+
+#include "gqla.h"
+#include "launch.h"
+#include "tc.h"
+
+namespace {
+
+// 32 MiB of split scratch per device that loads the library, held until the
+// process exits.
+constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array for the current device.  In host code
+// g_noalloc_scratch names a host-side stand-in, not device memory, so the
+// address is looked up once per device (with that device current) and cached.
+void* scratch_for_current_device(gqla_status* status) {
+  static std::mutex mu;
+  static void* cached[64] = {nullptr};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    *status = GQLA_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cached[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      *status = GQLA_ERR_CUDA;
+      return nullptr;
+    }
+    cached[dev] = ptr;
+  }
+  return cached[dev];
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+
+using namespace gqla;
+
+extern "C" gqla_status gqla_decode_gqa_noalloc(const gqla_dims* dims, const gqla_kv_layout* layout,
+                                               const void* q, const void* k_pool, const void* v_pool, void* out,
+                                               float* lse, int32_t num_splits, int32_t* dev_status,
+                                               void* stream) {
+  Problem p;
+  gqla_status s = make_problem(dims, layout, num_splits, GQLA_PATH_GQA, &p);
+  if (s != GQLA_OK) return s;
+  if (!q || !k_pool || !v_pool || !out) return GQLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out)) return GQLA_ERR_ALIGNMENT;
+  const bool tc = tc_gqa_supports(p);
+  if (!tc && !simt_supports(p, GQLA_PATH_GQA)) return GQLA_ERR_UNSUPPORTED;
+  const size_t need = ws_layout(p, GQLA_PATH_GQA, false, nullptr, nullptr);
+  if (need > kNoAllocScratchBytes) return GQLA_ERR_WORKSPACE;   // ask for fewer splits
+  void* scratch = nullptr;
+  if (need > 0) {
+    s = GQLA_OK;
+    scratch = scratch_for_current_device(&s);
+    if (!scratch) return s;
+  }
+  Workspace w;
+  ws_layout(p, GQLA_PATH_GQA, false, &w, (char*)scratch);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int S = p.plan.num_splits;
+  // Every split writes its whole partial (an empty split writes zeros and
+  // lse = -inf), so nothing left in the scratch by an earlier call is read.
+  cudaError_t e;
+  if (tc) e = tc_gqa_decode(p, q, k_pool, v_pool, S > 1 ? nullptr : out, S > 1 ? w.o_part : nullptr,
+                            S > 1 ? w.lse_part : lse, dev_status, st);
+  else e = simt_decode(p, GQLA_PATH_GQA, q, nullptr, k_pool, v_pool, S > 1 ? nullptr : out,
+                       S > 1 ? w.o_part : nullptr, S > 1 ? w.lse_part : lse, dev_status, st);
+  if (e == cudaSuccess && S > 1) e = combine(S, p.rows, p.d.d_v, w.o_part, w.lse_part, out, p.d.dtype, lse, st);
+  return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;
+}

@@ -31,6 +31,12 @@ struct Workspace {
   float* o_lat;    // absorb: combined latent outputs [rows, r]
 };
 
+// Validates dims/layout and builds the problem with its split plan.
+gqla_status make_problem(const gqla_dims* dims, const gqla_kv_layout* layout, int num_splits, gqla_path path,
+                         Problem* p);
+// The generic kernels keep a row's query and accumulator in registers.
+bool simt_supports(const Problem& p, gqla_path path);
+
 size_t ws_layout(const Problem& p, gqla_path path, bool tc, Workspace* ws, char* base);
 
 // ---- generic CUDA-core kernels (fp32 math; any supported dims) ----

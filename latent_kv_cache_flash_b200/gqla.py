@@ -55,6 +55,7 @@ def lib():
         L.gqla_expand_cache.argtypes = [pd, pl, P, P, P, P, P, I32, P, P]
         L.gqla_decode_absorb.argtypes = [pd, pl, P, P, P, P, P, P, I32, P, SZ, P, P]
         L.gqla_decode_gqa.argtypes = [pd, pl, P, P, P, P, P, I32, P, SZ, P, P]
+        L.gqla_decode_gqa_noalloc.argtypes = [pd, pl, P, P, P, P, P, I32, P, P]
         L.gqla_splitkv_combine.argtypes = [I32, I32, I32, P, P, P, ctypes.c_int, P, P]
         L.gqla_workspace_bytes.argtypes = [pd, pl, I32, ctypes.c_int]
         L.gqla_workspace_bytes.restype = SZ
@@ -66,7 +67,8 @@ def lib():
         L.gqla_status_string.restype = ctypes.c_char_p
         L.gqla_version.restype = ctypes.c_char_p
         L.gqla_launch_counter.restype = ctypes.c_uint64
-        for name in ("gqla_expand_cache", "gqla_decode_absorb", "gqla_decode_gqa", "gqla_splitkv_combine"):
+        for name in ("gqla_expand_cache", "gqla_decode_absorb", "gqla_decode_gqa", "gqla_decode_gqa_noalloc",
+                     "gqla_splitkv_combine"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -164,6 +166,16 @@ def gqla_decode_gqa(dims, layout, q, k_pool, v_pool, out, lse=None, num_splits=0
                               workspace.numel() * workspace.element_size(), _ptr(dev_status),
                               _stream(stream, q.device))
     _check(s, "gqla_decode_gqa")
+
+
+def gqla_decode_gqa_noalloc(dims, layout, q, k_pool, v_pool, out, lse=None, num_splits=0, dev_status=None,
+                            stream=None):
+    """gqla_decode_gqa with its split scratch in the library's own fixed device
+    array: no workspace, no allocation (see include/gqla.h for the limit)."""
+    s = lib().gqla_decode_gqa_noalloc(ctypes.byref(dims), ctypes.byref(layout), _ptr(q), _ptr(k_pool),
+                                      _ptr(v_pool), _ptr(out), _ptr(lse), int(num_splits), _ptr(dev_status),
+                                      _stream(stream, q.device))
+    _check(s, "gqla_decode_gqa_noalloc")
 
 
 def gqla_splitkv_combine(o_part, lse_part, out, lse_out=None, stream=None):
