@@ -201,24 +201,25 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ ours ---
-def kernel_sha():
+def kernel_sha(files):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "latent_kv_cache_flash_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in files:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel_name):
+def recorded_traffic(name):
+    """DRAM bytes per launch from the committed ncu record of this kernel, or
+    None when the kernel's sources changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        rec = json.load(open(p)).get(kernel_name)
+        rec = json.load(open(p)).get(name)
+        if not rec or rec.get("source_sha") != kernel_sha(rec["files"]):
+            return None
     except Exception:
-        return None
-    if not rec or rec.get("source_sha") != kernel_sha():
         return None
     return rec.get("bytes_per_launch")
 
@@ -228,9 +229,8 @@ def run_ours(args):
     import torch.distributed as dist
     from latent_kv_cache_flash_b200 import build, gqla, synth
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from latent_kv_cache_flash_b200 import multi
+    rank, local, world = multi.rank_info()
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU (no CPU fallback)")
     torch.cuda.set_device(local)
@@ -242,7 +242,7 @@ def run_ours(args):
     hbm, tf_burst, tf_sust, peak_src = load_peaks()
 
     wl = workload(args.sq)
-    wl.seed = wl.seed + rank
+    wl.seed = multi.rank_seed(wl.seed, rank)
     d = wl.dims
     inp = synth.make_inputs(wl, dev)
     dims = gqla.make_dims(d)
@@ -277,9 +277,7 @@ def run_ours(args):
         absorb()
         gqa()
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = multi.barrier
 
     def timed(fn, n):
         torch.cuda.synchronize()
@@ -291,12 +289,7 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return multi.max_over_ranks(e0.elapsed_time(e1), dev)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -355,7 +348,7 @@ def run_ours(args):
 
     alg = algorithmic(wl)
     tokens = B * d.s_q
-    value = world * tokens / (ms_step * 1e-3)
+    value = multi.job_tokens_per_s(tokens, 1, world, ms_step)
     # dominant kernel: the slower decode call of the step
     if ms_gqa >= ms_absorb:
         name, ms_dom, bytes_dom = "gqla_decode_gqa", ms_gqa, alg["gqa_bytes"]
