@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
+    ap.add_argument("--sweep", choices=["crossover", "context", "ragged"],
+                    help="instead of the headline line, time both decode paths over a workload sweep "
+                         "(one JSON line per point)")
     return ap.parse_args()
 
 
@@ -418,10 +421,95 @@ def run_ours(args):
     return 0
 
 
+def time_paths(inp, reps, hbm, tf_burst, expand=True):
+    """Device time of one absorb call and one GQA call on resident inputs.
+    With expand=False the per-group pools are filled with seeded random bf16
+    instead of the expansion (decode time does not depend on the values)."""
+    import torch
+    from latent_kv_cache_flash_b200 import gqla, synth
+    d = inp.dims
+    dev = inp.q.device
+    dims = gqla.make_dims(d)
+    lay = gqla.make_layout(inp.seq_lens, inp.max_seq_len, inp.wl.page_size,
+                           inp.capacity if inp.wl.page_size == 0 else 0, inp.block_table, inp.num_pages)
+    ks, vs = synth.expanded_pool_shapes(inp)
+    if expand:
+        kp = torch.empty(ks, dtype=d.torch_dtype, device=dev)
+        vp = torch.empty(vs, dtype=d.torch_dtype, device=dev)
+        gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp)
+    else:
+        g = torch.Generator(device=dev)
+        g.manual_seed(1)
+        kp = synth._randn_chunked(ks, g, dev, d.torch_dtype)
+        vp = synth._randn_chunked(vs, g, dev, d.torch_dtype)
+    B = inp.wl.batch
+    out = torch.empty((B, d.s_q, d.n_h, d.d_v), dtype=d.torch_dtype, device=dev)
+    lse = torch.empty((B, d.s_q, d.n_h), device=dev)
+    ws_a = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_ABSORB, dev)
+    ws_g = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_GQA, dev)
+    res = {}
+    lens = inp.seq_lens_host
+    T = sum(lens)
+    keys = sum(sum(L - d.s_q + i + 1 for i in range(d.s_q)) for L in lens)
+    work = {"absorb": (2 * T * (d.r + d.d_rope), d.n_h * keys * 2 * (2 * d.r + d.d_rope)),
+            "gqa": (2 * T * d.G * (d.d_qk + d.d_v), d.n_h * keys * 2 * (d.d_qk + d.d_v))}
+    calls = {"absorb": lambda: gqla.gqla_decode_absorb(dims, lay, inp.q, inp.latent, inp.W_uk, inp.W_uv, out, lse,
+                                                        0, ws_a),
+             "gqa": lambda: gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out, lse, 0, ws_g)}
+    for name, fn in calls.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        nbytes, flops = work[name]
+        t_hbm, t_tc = nbytes / (hbm * 1e9), flops / (tf_burst * 1e12)
+        res[name] = {"ms": ms, "tokens_per_s": B * d.s_q / (ms * 1e-3), "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                     "roofline_frac": max(t_hbm, t_tc) / (ms * 1e-3), "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+                     "tflops": flops / (ms * 1e-3) / 1e12,
+                     "splits": gqla.gqla_num_splits(dims, lay, 0, 0 if name == "absorb" else 1)}
+    del kp, vp
+    return res
+
+
+def run_sweep(args):
+    """Both decode paths over the crossover, context or ragged workloads."""
+    import torch
+    from latent_kv_cache_flash_b200 import build, synth
+    build.build()
+    hbm, tf_burst, _, _ = load_peaks()
+    if args.sweep == "crossover":
+        points = [synth.crossover(G, s_q) for G in (1, 2, 4, 8, 16, 32, 128) for s_q in (1, 2, 4)]
+    elif args.sweep == "context":
+        points = [synth.dsv3(seq_len=L, s_q=s_q) for L in (8192, 16384, 32768, 65536) for s_q in (1, 2)]
+    else:
+        points = [synth.ragged_paged()]
+    for wl in points:
+        inp = synth.make_inputs(wl, "cuda")
+        res = time_paths(inp, max(5, args.steps // 10), hbm, tf_burst, expand=False)
+        d = wl.dims
+        line = {"sweep": args.sweep, "workload": wl.name, "G": d.G, "s_q": d.s_q, "batch": wl.batch,
+                "seq_len": wl.seq_len if wl.ragged is None else "ragged %d..%d" % wl.ragged,
+                "page_size": wl.page_size, "absorb": res["absorb"], "gqa": res["gqa"],
+                "faster": "absorb" if res["absorb"]["ms"] < res["gqa"]["ms"] else "gqa",
+                "pools": "expanded pools filled with seeded random bf16 (decode timing only)"}
+        print(json.dumps(line), flush=True)
+        del inp
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args)
 
 

@@ -53,13 +53,16 @@ __device__ __forceinline__ uint64_t global_ns() {
 // try_wait (which itself suspends the thread for a short while) and gives up
 // after about kWaitLimitNs of wall time.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+    if ((i & 1023u) == 0 && global_ns() - t0 > limit_ns) return false;
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // -------------------------------------------------------------------- TMA

@@ -27,7 +27,7 @@ bool gemm_combine_up_supports(const Problem& p);
 cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const float* lse_part, const void* W_uv,
                            void* out, float* lse_out, __nv_bfloat16* o_lat, cudaStream_t s);
 
-// Cache expansion GEMM (tc_gemm.cu).
+// Cache expansion GEMM on tcgen05 (tc_expand.cu).
 bool tc_expand_supports(const Problem& p);
 cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, const void* W_uv, void* k_pool,
                       void* v_pool, int tail, int32_t* st, cudaStream_t s);

@@ -1,0 +1,330 @@
+// Per-group cache expansion on the 5th-generation tensor cores (tcgen05).
+//
+// The GQA path runs over a per-group expanded cache ("GQLA" chatpaper.ai
+// Abstract): for every token t and group g,
+//     K[t, g] = [ c_t W_uk^g ; k_rope_t ],   V[t, g] = c_t W_uv^g.
+// Per group this is one dense GEMM  C = X [T x 512] * [W_uk^g | W_uv^g]
+// [512 x 256], so it runs as a persistent tcgen05 GEMM:
+//  * work item = (128-token tile, group), group index fastest, so the G items
+//    that share a latent tile run at the same time and L2 serves the re-reads;
+//  * warp 0 streams K-chunks of 64 (A: 128 tokens x 64, two 64-row TMA boxes
+//    so that a tile may span two pages; B: 64 rows x 256 columns of the two
+//    weight matrices) into a 4-stage mbarrier ring;
+//  * warp 1 issues 4 tcgen05.mma (M=128, N=256, K=16; A K-major, B MN-major)
+//    per chunk into one of two TMEM accumulators (2 x 256 columns);
+//  * warps 2-5 drain an accumulator (tcgen05.ld, one token row per thread),
+//    round to bf16 and write the K and V rows, and copy the shared RoPE key.
+// Tiles start on a 64-token boundary; rows outside [first token, L) of the
+// sequence are computed but not written.
+#include "ptx.cuh"
+#include "tc.h"
+
+namespace gqla {
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kR = 512, kDn = 128, kDv = 128, kDr = 64, kE = kR + kDr;
+constexpr int kTM = 128;                          // tokens per tile
+constexpr int kN = kDn + kDv;                     // 256 outputs per group
+constexpr int kKC = 64;                           // K per stage
+constexpr int kStages = 4;
+constexpr int kABytes = kTM * 128;                // 16 KB
+constexpr int kBBox = kKC * 128;                  // 8 KB: 64 K-rows x 64 columns
+constexpr int kBBytes = 4 * kBBox;                // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;    // 48 KB
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kThreads = 6 * 32;
+
+struct ExpandParams {
+  KvLayout ly;
+  bf16* kp;
+  bf16* vp;
+  const bf16* latent;
+  int G;
+  int tail;          // > 0: only the newest `tail` tokens of each sequence
+  int tps;           // tiles per sequence
+  long long n_items; // batch * tps * G
+  int32_t* st;
+};
+
+// Tile j of sequence b: first token t0 (64-aligned) and the token range
+// [t_lo, t_hi) that is written.  Returns false when the item is empty.
+__device__ __forceinline__ bool item_tile(const ExpandParams& p, int b, int j, int* t0, int* t_lo, int* t_hi,
+                                          bool report = false) {
+  const KvLayout& ly = p.ly;
+  const int L = ly.seq_lens[b];
+  const bool bad = L < 1 || L > ly.max_seq_len ||
+                   (ly.page_size == 0 ? L > ly.capacity : (L + ly.page_size - 1) / ly.page_size > ly.mbps);
+  if (bad) {
+    if (report && j == 0) flag_status(p.st, L < 1 ? GQLA_DEV_SHORT_SEQ : GQLA_DEV_OVERFLOW);
+    return false;
+  }
+  const int start = p.tail > 0 ? max(0, L - p.tail) : 0;
+  *t0 = (start / 64) * 64 + j * kTM;
+  *t_lo = start;
+  *t_hi = L;
+  return *t0 < L;
+}
+
+// Pool row of the first token of a 64-token half tile (valid pages only;
+// rows past the sequence read any in-pool row and are never written).
+__device__ __forceinline__ int half_row(const KvLayout& ly, int b, int t, int L) {
+  if (ly.page_size == 0) return (int)((long long)b * ly.capacity + t);
+  const int nb = (L + ly.page_size - 1) / ly.page_size;
+  const int blk = t / ly.page_size;
+  if (blk >= nb) return 0;
+  const int page = ly.block_table[(long long)b * ly.mbps + blk];
+  if (page < 0 || page >= ly.num_pages) return 0;
+  return page * ly.page_size + (t % ly.page_size);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    expand_tc_kernel(const __grid_constant__ CUtensorMap lat_map, const __grid_constant__ CUtensorMap uk_map,
+                     const __grid_constant__ CUtensorMap uv_map, const ExpandParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], acc_full[2], acc_empty[2], drain;
+  __shared__ uint32_t tmem_base_sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(&full_bar[s], 1);
+      ptx::mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&acc_full[a], 1);
+      ptx::mbar_init(&acc_empty[a], 4);
+    }
+    ptx::mbar_init(&drain, 1);
+    ptx::fence_barrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&tmem_base_sh, kTmemCols);
+    ptx::tmem_relinquish();
+    ptx::tc_fence_before();
+  }
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int G = p.G;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&lat_map);
+      ptx::prefetch_tmap(&uk_map);
+      ptx::prefetch_tmap(&uv_map);
+      long long it = 0;
+      bool ok = true;
+      for (long long item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int g = (int)(item % G);
+        const long long bt = item / G;
+        const int b = (int)(bt / p.tps), j = (int)(bt % p.tps);
+        int t0, tlo, thi;
+        if (!item_tile(p, b, j, &t0, &tlo, &thi, g == 0)) continue;
+        const int row0 = half_row(p.ly, b, t0, thi), row1 = half_row(p.ly, b, t0 + 64, thi);
+        for (int kc = 0; kc < kR / kKC; ++kc, ++it) {
+          const int s = (int)(it % kStages);
+          const long long k = it / kStages;
+          if (k > 0 && !ptx::mbar_wait(&empty_bar[s], (uint32_t)((k - 1) & 1))) {
+            flag_status(p.st, GQLA_DEV_TIMEOUT);
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStageBytes;
+          ptx::mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
+          ptx::tma_load_2d(st, &lat_map, &full_bar[s], kKC * kc, row0);
+          ptx::tma_load_2d(st + kABytes / 2, &lat_map, &full_bar[s], kKC * kc, row1);
+          uint8_t* bs = st + kABytes;
+          const int wrow = g * kR + kKC * kc;
+          ptx::tma_load_2d(bs + 0 * kBBox, &uk_map, &full_bar[s], 0, wrow);
+          ptx::tma_load_2d(bs + 1 * kBBox, &uk_map, &full_bar[s], 64, wrow);
+          ptx::tma_load_2d(bs + 2 * kBBox, &uv_map, &full_bar[s], 0, wrow);
+          ptx::tma_load_2d(bs + 3 * kBBox, &uv_map, &full_bar[s], 64, wrow);
+        }
+      }
+      // no copy may still be landing when the CTA retires
+      for (long long i = it > kStages ? it - kStages : 0; i < it; ++i)
+        ptx::mbar_wait(&full_bar[i % kStages], (uint32_t)((i / kStages) & 1));
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_bf16(kTM, kN, false, true);
+      const uint32_t base = ptx::smem_u32(smem);
+      long long it = 0, li = 0;
+      bool ok = true;
+      for (long long item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int g = (int)(item % G);
+        const long long bt = item / G;
+        const int b = (int)(bt / p.tps), j = (int)(bt % p.tps);
+        int t0, tlo, thi;
+        (void)g;
+        if (!item_tile(p, b, j, &t0, &tlo, &thi)) continue;
+        const int ab = (int)(li & 1);
+        if (li >= 2 && !ptx::mbar_wait(&acc_empty[ab], (uint32_t)(((li >> 1) - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        const uint32_t d = tmem + (uint32_t)(ab * kN);
+        for (int kc = 0; kc < kR / kKC; ++kc, ++it) {
+          const int s = (int)(it % kStages);
+          if (!ptx::mbar_wait(&full_bar[s], (uint32_t)((it / kStages) & 1))) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a_addr = base + s * kStageBytes;
+          const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kKC / 16; ++kk) {
+            const uint64_t ad = ptx::umma_desc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = ptx::umma_desc_sw128(b_addr + kk * 16 * 128, kBBox, 1024);
+            ptx::umma_bf16(d, ad, bd, idesc, (kc | kk) != 0);
+          }
+          ptx::umma_commit(&empty_bar[s]);
+        }
+        if (!ok) break;
+        ptx::umma_commit(&acc_full[ab]);
+        ++li;
+      }
+      if (!ok) flag_status(p.st, GQLA_DEV_TIMEOUT);
+      ptx::umma_commit(&drain);
+      ptx::mbar_wait(&drain, 0);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int qd = warp & 3;                   // TMEM lane quarter
+    const int r = 32 * qd + lane;              // tile row = token offset
+    const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+    long long li = 0;
+    bool ok = true;
+    for (long long item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+      const int g = (int)(item % G);
+      const long long bt = item / G;
+      const int b = (int)(bt / p.tps), j = (int)(bt % p.tps);
+      int t0, tlo, thi;
+      if (!item_tile(p, b, j, &t0, &tlo, &thi)) continue;
+      const int ab = (int)(li & 1);
+      if (ok) ok = ptx::mbar_wait(&acc_full[ab], (uint32_t)((li >> 1) & 1));
+      ok = __all_sync(0xffffffffu, ok);
+      const int t = t0 + r;
+      const bool write = ok && t >= tlo && t < thi;
+      long long row = 0;
+      if (write) row = half_row(p.ly, b, t0 + (r & ~63), thi) + (r & 63);
+      if (ok) {
+        ptx::tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < kN / 32; ++c) {
+          uint32_t v[32];
+          ptx::tmem_ld32(tl + (uint32_t)(ab * kN + 32 * c), v);
+          ptx::tmem_ld_wait();
+          if (write) {
+            bf16* dst = c < kDn / 32 ? p.kp + (row * G + g) * (kDn + kDr) + 32 * c
+                                     : p.vp + (row * G + g) * kDv + 32 * (c - kDn / 32);
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 w;
+              w.x = ptx::pack_bf16(__uint_as_float(v[e + 0]), __uint_as_float(v[e + 1]));
+              w.y = ptx::pack_bf16(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+              w.z = ptx::pack_bf16(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+              w.w = ptx::pack_bf16(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+              *reinterpret_cast<uint4*>(dst + e) = w;
+            }
+          }
+        }
+        if (write) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.latent + row * kE + kR);
+          uint4* dst = reinterpret_cast<uint4*>(p.kp + (row * G + g) * (kDn + kDr) + kDn);
+#pragma unroll
+          for (int e = 0; e < kDr / 8; ++e) dst[e] = src[e];
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&acc_empty[ab]);
+      ++li;
+    }
+    if (!ok && lane == 0) flag_status(p.st, GQLA_DEV_TIMEOUT);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)f;
+  }
+  return fn;
+}
+
+bool map_2d(CUtensorMap* map, const void* base, long long cols, long long rows, long long pitch, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)pitch * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tc_expand_supports(const Problem& p) {
+  const auto& d = p.d;
+  if (d.dtype != GQLA_BF16 || d.r != kR || d.d_nope != kDn || d.d_v != kDv || d.d_rope != kDr) return false;
+  if (p.ly.page_size != 0 && p.ly.page_size % 64 != 0) return false;
+  const long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
+                                              : (long long)p.ly.num_pages * p.ly.page_size;
+  if (nrows + 128 >= (1LL << 31)) return false;
+  return true;
+}
+
+cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, const void* W_uv, void* k_pool,
+                      void* v_pool, int tail, int32_t* st, cudaStream_t s) {
+  const auto& d = p.d;
+  const long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
+                                              : (long long)p.ly.num_pages * p.ly.page_size;
+  CUtensorMap lat_map, uk_map, uv_map;
+  if (!map_2d(&lat_map, latent, kE, nrows, kE, 64) || !map_2d(&uk_map, W_uk, kDn, (long long)d.G * kR, kDn, kKC) ||
+      !map_2d(&uv_map, W_uv, kDv, (long long)d.G * kR, kDv, kKC))
+    return cudaErrorInvalidValue;
+  ExpandParams prm;
+  prm.ly = p.ly;
+  prm.kp = (bf16*)k_pool;
+  prm.vp = (bf16*)v_pool;
+  prm.latent = (const bf16*)latent;
+  prm.G = d.G;
+  const int span = tail > 0 ? (tail < p.ly.max_seq_len ? tail : p.ly.max_seq_len) : p.ly.max_seq_len;
+  prm.tail = tail > 0 ? span : 0;
+  prm.tps = (span + 63 + kTM - 1) / kTM;
+  prm.n_items = (long long)p.ly.batch * prm.tps * d.G;
+  prm.st = st;
+  cudaError_t e = ensure_smem_limit((const void*)expand_tc_kernel, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const long long grid = prm.n_items < num_sms() ? prm.n_items : num_sms();
+  if (grid < 1) return cudaSuccess;
+  expand_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(lat_map, uk_map, uv_map, prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace gqla

@@ -3,10 +3,7 @@
 //  * absorb_q:      q~[row] = W_uk^g q_nope[row]          (per group, r outputs)
 //  * combine_lat + up_proj: LSE merge of the split partials of the latent
 //                   output (bf16), then out[row] = o_lat[row] W_uv^g
-//  * expand:        K[t,g] = [c_t W_uk^g ; k_rope_t], V[t,g] = c_t W_uv^g
-//                   (the GQA path's per-group expanded cache, for all tokens
-//                   or for the newest `tail` tokens of every sequence)
-// All three read their row-major operands through ldmatrix from padded shared
+// They read their row-major operands through ldmatrix from padded shared
 // memory; the weight operand is shared by every row of a group.
 #include <math.h>
 
@@ -243,131 +240,6 @@ __global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict
   }
 }
 
-// --------------------------------------------------------------- expand
-// CTA: 64 tokens x 64 outputs of group g (quarter q of its 256 outputs: q = 0,1
-// key-nope through W_uk^g, q = 2,3 values through W_uv^g); 4 warps of 16 rows.
-// K = 512 in 64-wide chunks, double-buffered with cp.async.  Quarter 0 also
-// copies the shared RoPE key into the group's key.
-constexpr int kExR = 512, kExDn = 128, kExDv = 128, kExDr = 64, kExE = kExR + kExDr;
-constexpr int kExT = 64, kExKC = 64, kExN = 64;
-constexpr int kExApitch = (kExKC + 8) * 2;                 // 144 B
-constexpr int kExBpitch = (kExN + 8) * 2;                  // 144 B
-constexpr int kExAbytes = kExT * kExApitch;
-constexpr int kExBbytes = kExKC * kExBpitch;
-constexpr size_t kExSmem = 2 * (size_t)(kExAbytes + kExBbytes);
-
-__global__ void __launch_bounds__(128) expand_mma_kernel(KvLayout ly, const bf16* __restrict__ latent,
-                                                         const bf16* __restrict__ W_uk,
-                                                         const bf16* __restrict__ W_uv, bf16* __restrict__ kp,
-                                                         bf16* __restrict__ vp, int G, int tail, int blocks_per_seq,
-                                                         long long n_tiles, int32_t* st) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  __shared__ long long srow[kExT];
-  // blockIdx.x = (group, quarter) fastest so that the 4*G CTAs sharing a
-  // token tile run together and its latent rows are read from DRAM once;
-  // token tiles stride over blockIdx.y
-  const int g = blockIdx.x >> 2, quarter = blockIdx.x & 3;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool is_k = quarter < 2;
-  const bf16* Wsrc = is_k ? W_uk + (size_t)g * kExR * kExDn + quarter * kExN
-                          : W_uv + (size_t)g * kExR * kExDv + (quarter - 2) * kExN;
-  const int wld = is_k ? kExDn : kExDv;
-  const uint32_t base = ptx::smem_u32(sm);
-  for (long long tile = blockIdx.y; tile < n_tiles; tile += gridDim.y) {
-    // which token each tile row holds (pool row, or -1)
-    __syncthreads();
-    if (threadIdx.x < kExT) {
-      long long row = -1;
-      int b, t;
-      if (tail > 0) {
-        const long long idx = tile * kExT + threadIdx.x;
-        b = (int)(idx / tail);
-        t = b < ly.batch ? ly.seq_lens[b] - tail + (int)(idx % tail) : -1;
-      } else {
-        b = (int)(tile / blocks_per_seq);
-        t = (int)(tile % blocks_per_seq) * kExT + threadIdx.x;
-      }
-      if (b < ly.batch) {
-        const int L = ly.seq_lens[b];
-        const bool bad = L < 1 || L > ly.max_seq_len ||
-                         (ly.page_size == 0 ? L > ly.capacity : (L + ly.page_size - 1) / ly.page_size > ly.mbps);
-        const bool reporter = g == 0 && quarter == 0 &&
-                              (tail > 0 ? (int)((tile * kExT + threadIdx.x) % tail) == 0 : t == 0);
-        if (bad) {
-          if (reporter) flag_status(st, L < 1 ? GQLA_DEV_SHORT_SEQ : GQLA_DEV_OVERFLOW);
-        } else if (t >= 0 && t < L) {
-          row = token_row(ly, b, t, (g == 0 && quarter == 0) ? st : nullptr);
-        }
-      }
-      srow[threadIdx.x] = row;
-    }
-    __syncthreads();
-    auto load_chunk = [&](int kc, int buf) {
-      const uint32_t a = base + buf * (kExAbytes + kExBbytes);
-      const uint32_t bb = a + kExAbytes;
-      for (int i = threadIdx.x; i < kExT * (kExKC / 8); i += blockDim.x) {
-        const int tt = i / (kExKC / 8), c = i % (kExKC / 8);
-        const long long row = srow[tt];
-        cp_async16(a + tt * kExApitch + c * 16, latent + (row < 0 ? 0 : row) * kExE + kc + c * 8, row >= 0);
-      }
-      for (int i = threadIdx.x; i < kExKC * (kExN / 8); i += blockDim.x) {
-        const int kk = i / (kExN / 8), c = i % (kExN / 8);
-        cp_async16(bb + kk * kExBpitch + c * 16, Wsrc + (size_t)(kc + kk) * wld + c * 8, true);
-      }
-      cp_async_commit();
-    };
-    float acc[kExN / 8][4];
-#pragma unroll
-    for (int n = 0; n < kExN / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-    load_chunk(0, 0);
-    for (int c = 0; c < kExR / kExKC; ++c) {
-      if (c + 1 < kExR / kExKC) {
-        load_chunk((c + 1) * kExKC, (c + 1) & 1);
-        cp_async_wait1();
-      } else {
-        cp_async_wait0();
-      }
-      __syncthreads();
-      const uint32_t a = base + (c & 1) * (kExAbytes + kExBbytes);
-      const uint32_t bb = a + kExAbytes;
-#pragma unroll
-      for (int k0 = 0; k0 < kExKC; k0 += 16) {
-        uint32_t af[4];
-        ldsm_a(a, kExApitch, warp * 16, k0, af);
-#pragma unroll
-        for (int np = 0; np < kExN / 16; ++np) {
-          uint32_t b[4];
-          ldsm_b_kn(bb, kExBpitch, np * 16, k0, b);
-          ptx::mma_bf16_16816(acc[2 * np], af, b[0], b[1]);
-          ptx::mma_bf16_16816(acc[2 * np + 1], af, b[2], b[3]);
-        }
-      }
-      __syncthreads();
-    }
-    const int gid = lane >> 2, tig = lane & 3;
-    constexpr int kDqk = kExDn + kExDr;
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      const long long row = srow[warp * 16 + gid + 8 * h2];
-      if (row < 0) continue;
-      bf16* dst = is_k ? kp + (row * G + g) * kDqk + quarter * kExN : vp + (row * G + g) * kExDv + (quarter - 2) * kExN;
-#pragma unroll
-      for (int n = 0; n < kExN / 8; ++n)
-        *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * tig) = ptx::pack_bf16(acc[n][2 * h2], acc[n][2 * h2 + 1]);
-    }
-    if (quarter == 0) {
-      // the shared RoPE key is copied into every group's key
-      for (int i = threadIdx.x; i < kExT * (kExDr / 8); i += blockDim.x) {
-        const int tt = i / (kExDr / 8), c = i % (kExDr / 8);
-        const long long row = srow[tt];
-        if (row < 0) continue;
-        *reinterpret_cast<uint4*>(kp + (row * G + g) * kDqk + kExDn + c * 8) =
-            *reinterpret_cast<const uint4*>(latent + row * kExE + kExR + c * 8);
-      }
-    }
-  }
-}
-
 }  // namespace
 
 bool gemm_absorb_q_supports(const Problem& p) {
@@ -405,27 +277,6 @@ cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const f
   if (e != cudaSuccess) return e;
   dim3 grid((rows_g + kUpRows - 1) / kUpRows, d.G);
   up_proj_mma_kernel<<<grid, 128, kUpSmem, s>>>(o_lat, (const bf16*)W_uv, (bf16*)out, rows_g, d.n_h, p.m);
-  count_launch();
-  return cudaGetLastError();
-}
-
-bool tc_expand_supports(const Problem& p) {
-  const auto& d = p.d;
-  return d.dtype == GQLA_BF16 && d.r == kExR && d.d_nope == kExDn && d.d_v == kExDv && d.d_rope == kExDr;
-}
-
-cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, const void* W_uv, void* k_pool,
-                      void* v_pool, int tail, int32_t* st, cudaStream_t s) {
-  const int span = tail > 0 ? (tail < p.ly.max_seq_len ? tail : p.ly.max_seq_len) : p.ly.max_seq_len;
-  const int bps = (span + kExT - 1) / kExT;
-  long long gx = tail > 0 ? ((long long)p.ly.batch * span + kExT - 1) / kExT : (long long)p.ly.batch * bps;
-
-  cudaError_t e = ensure_smem_limit((const void*)expand_mma_kernel, (int)kExSmem);
-  if (e != cudaSuccess) return e;
-  if (gx < 1) return cudaSuccess;
-  dim3 grid(p.d.G * 4, (unsigned)(gx < 65535 ? gx : 65535));
-  expand_mma_kernel<<<grid, 128, kExSmem, s>>>(p.ly, (const bf16*)latent, (const bf16*)W_uk, (const bf16*)W_uv,
-                                               (bf16*)k_pool, (bf16*)v_pool, p.d.G, tail > 0 ? span : 0, bps, gx, st);
   count_launch();
   return cudaGetLastError();
 }
