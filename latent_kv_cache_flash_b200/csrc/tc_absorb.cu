@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sKV = smem + kQBytes;
   uint8_t* sP = sKV + kStages * kStageBytes;
   __shared__ __align__(8) uint64_t q_full, p_full, pv_done, qk_drain, pv_drain;
-  __shared__ __align__(8) uint64_t kv_full[kStages][kChunks], kv_empty[kStages], s_full[2], s_free[2];
+  __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(&qk_drain, 1);
     ptx::mbar_init(&pv_drain, 1);
     for (int s = 0; s < kStages; ++s) {
-      for (int c = 0; c < kChunks; ++c) ptx::mbar_init(&kv_full[s][c], 1);
+      ptx::mbar_init(&kv_full[s], 1);
       ptx::mbar_init(&kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -134,18 +134,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*(volatile int*)&abort_flag) break;
         const int row0 = (int)token_row(p.ly, b, t_begin + j * kTk, nullptr);
         uint8_t* dst = sKV + s * kStageBytes;
-        // one barrier per 64-column chunk: QK starts on the first chunk while
-        // the rest of the tile is still arriving
-        for (int c = 0; c < kChunks; ++c) {
-          ptx::mbar_arrive_expect_tx(&kv_full[s][c], kKVChunk);
-          ptx::tma_load_2d(dst + c * kKVChunk, &kv_map, &kv_full[s][c], 64 * c, row0);
-        }
+        ptx::mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
+        for (int c = 0; c < kChunks; ++c) ptx::tma_load_2d(dst + c * kKVChunk, &kv_map, &kv_full[s], 64 * c, row0);
         issued = j + 1;
       }
       // no copy may still be landing in shared memory when the CTA retires
       ptx::mbar_wait(&q_full, 0);
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-        for (int c = 0; c < kChunks; ++c) ptx::mbar_wait(&kv_full[j % kStages][c], (j / kStages) & 1);
+        ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------- QK issuer, TMEM owner
@@ -155,23 +151,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = ptx::mbar_wait(&q_full, 0);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kStages, sb = j & 1;
-        if (j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
+        ok = ptx::mbar_wait(&kv_full[s], (j / kStages) & 1);
+        if (ok && j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
         if (!ok) break;
+        ptx::tc_fence_after();
         const uint32_t d = tmem + kSCol + (uint32_t)kTk * sb;
         const uint32_t st_addr = kv_addr + s * kStageBytes;
-        for (int c = 0; ok && c < kChunks; ++c) {
-          ok = ptx::mbar_wait(&kv_full[s][c], (j / kStages) & 1);
-          if (!ok) break;
-          ptx::tc_fence_after();
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const uint32_t kin = k4 * 32;
-            const uint64_t a = ptx::umma_desc_sw128(q_addr + c * kQChunk + kin, 16, 1024);
-            const uint64_t bd = ptx::umma_desc_sw128(st_addr + c * kKVChunk + kin, 16, 1024);
-            ptx::umma_bf16(d, a, bd, idesc_qk, (c | k4) != 0);
-          }
+        for (int kk = 0; kk < kE / 16; ++kk) {
+          const uint32_t koff = (kk >> 2), kin = (kk & 3) * 32;
+          const uint64_t a = ptx::umma_desc_sw128(q_addr + koff * kQChunk + kin, 16, 1024);
+          const uint64_t bd = ptx::umma_desc_sw128(st_addr + koff * kKVChunk + kin, 16, 1024);
+          ptx::umma_bf16(d, a, bd, idesc_qk, kk > 0);
         }
-        if (!ok) break;
         ptx::umma_commit(&s_full[sb]);
       }
       if (!ok) {
