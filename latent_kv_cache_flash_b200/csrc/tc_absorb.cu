@@ -12,14 +12,16 @@
 // One CTA per (key-range split, sequence, block of 64 rows):
 //  * warp 0 loads the absorbed-query tile once (64 x 576, 72 KB) and streams
 //    64-token latent tiles (72 KB) with TMA into a 2-stage mbarrier ring;
-//  * warp 1 owns 512 TMEM columns and issues S = Q~ C^T as 36 tcgen05.mma
-//    (M=64, N=64, K=16) into a double-buffered S in TMEM; warp 6 issues
+//  * warps 1 and 7 issue S = Q~ C^T as 36 tcgen05.mma (M=64, N=64, K=16),
+//    split along K into two double-buffered S halves in TMEM (one issuing
+//    thread cannot keep up with such small MMAs); warp 1 owns the 512 TMEM
+//    columns; warp 6 issues
 //    O += P C[:, :512] as 8 tcgen05.mma (M=64, N=256, K=16), reading the same
 //    latent tile as an MN-major B operand.  Two issuing threads keep the
 //    stage release (after PV) independent of the next tile's QK issue;
 //  * the M=64 accumulator uses 16 of every 32 TMEM lanes, so the two 256-wide
 //    halves of O sit interleaved at lane offsets 0 and 16 of the same 256
-//    columns; the two S buffers take columns 256..383;
+//    columns; the S halves and buffers take columns 256..511;
 //  * warps 2-5 read S rows from TMEM, run the online softmax in the log2
 //    domain with lazy rescaling (O is only rescaled when a row max grows by
 //    more than 2^8), write P (bf16) to shared memory, and in the end scale O
@@ -49,8 +51,9 @@ constexpr int kStageBytes = kChunks * kKVChunk;      // 36864
 constexpr int kPBytes = kM * 128;                    // 64 rows x 64 tokens (bf16)
 constexpr size_t kSmemBytes = (size_t)kQBytes + (size_t)kStages * kStageBytes + kPBytes + 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol = 256;                  // two S buffers of kTk columns
-constexpr int kThreads = 7 * 32;
+constexpr uint32_t kSCol = 256;                  // S buffers: [half a|b][buffer 0|1] x kTk columns
+constexpr int kQkSplit = 18;                     // k-steps (of 36) issued by the first QK warp
+constexpr int kThreads = 8 * 32;
 constexpr float kRescaleLog2 = 8.f;
 
 struct AbsorbParams {
@@ -74,7 +77,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + kQBytes;
   uint8_t* sP = sKV + kStages * kStageBytes;
-  __shared__ __align__(8) uint64_t q_full, p_full, pv_done, qk_drain, pv_drain;
+  __shared__ __align__(8) uint64_t q_full, p_full, pv_done, qk_drain[2], pv_drain;
   __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -87,14 +90,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(&q_full, 1);
     ptx::mbar_init(&p_full, 4);
     ptx::mbar_init(&pv_done, 1);
-    ptx::mbar_init(&qk_drain, 1);
+    ptx::mbar_init(&qk_drain[0], 1);
+    ptx::mbar_init(&qk_drain[1], 1);
     ptx::mbar_init(&pv_drain, 1);
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(&kv_full[s], 1);
       ptx::mbar_init(&kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(&s_full[s], 1);
+      ptx::mbar_init(&s_full[s], 2);   // one commit from each QK issuer
       ptx::mbar_init(&s_free[s], 4);
     }
     abort_flag = 0;
@@ -143,11 +147,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
         ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1);
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------- QK issuer, TMEM owner
+  } else if (warp == 1 || warp == 7) {
+    // ------------------------------------------------------- QK issuers
+    // One tcgen05.mma costs its issuing thread about as much time as a small
+    // (N=64) MMA takes to run, so two warps issue the 36 QK k-steps: warp 1
+    // k-steps [0, kQkSplit) into S half a, warp 7 the rest into S half b; the
+    // softmax adds the halves.  Warp 1 also owns the TMEM allocation.
+    const int half_q = warp == 7 ? 1 : 0;
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = ptx::idesc_bf16(kM, kTk, false, false);
       const uint32_t q_addr = ptx::smem_u32(sQ), kv_addr = ptx::smem_u32(sKV);
+      const int k_lo = half_q ? kQkSplit : 0, k_hi = half_q ? kE / 16 : kQkSplit;
       bool ok = ptx::mbar_wait(&q_full, 0);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kStages, sb = j & 1;
@@ -155,14 +165,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t d = tmem + kSCol + (uint32_t)kTk * sb;
+        const uint32_t d = tmem + kSCol + (uint32_t)kTk * (2 * half_q + sb);
         const uint32_t st_addr = kv_addr + s * kStageBytes;
-#pragma unroll
-        for (int kk = 0; kk < kE / 16; ++kk) {
+        for (int kk = k_lo; kk < k_hi; ++kk) {
           const uint32_t koff = (kk >> 2), kin = (kk & 3) * 32;
           const uint64_t a = ptx::umma_desc_sw128(q_addr + koff * kQChunk + kin, 16, 1024);
           const uint64_t bd = ptx::umma_desc_sw128(st_addr + koff * kKVChunk + kin, 16, 1024);
-          ptx::umma_bf16(d, a, bd, idesc_qk, kk > 0);
+          ptx::umma_bf16(d, a, bd, idesc_qk, kk > k_lo);
         }
         ptx::umma_commit(&s_full[sb]);
       }
@@ -171,8 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicExch(&abort_flag, 1);
       }
       // every issued MMA has finished before TMEM is released
-      ptx::umma_commit(&qk_drain);
-      ptx::mbar_wait(&qk_drain, 0);
+      ptx::umma_commit(&qk_drain[half_q]);
+      ptx::mbar_wait(&qk_drain[half_q], 0);
     }
   } else if (warp == 6) {
     // ---------------------------------------------------------- PV issuer
@@ -229,9 +238,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sv[kTk];
       if (ok) {
         ptx::tc_fence_after();
+        uint32_t sb2[32];
         ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * sb, sv);
         ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * sb + 32u, sv + 32);
+        ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * (2 + sb), sb2);
         ptx::tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) sv[t] = __float_as_uint(__uint_as_float(sv[t]) + __uint_as_float(sb2[t]));
+        ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * (2 + sb) + 32u, sb2);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+          sv[32 + t] = __float_as_uint(__uint_as_float(sv[32 + t]) + __uint_as_float(sb2[t]));
       }
       ptx::tc_fence_before();
       __syncwarp();

@@ -238,3 +238,35 @@ def test_ragged_paged_full_size():
     for path in ("absorb", "gqa"):
         out, lse = H.run_decode(inp, path)
         H.check_units(inp, out, lse, H.sample_units(inp, 4, seed=8), "ragged paged %s" % path)
+
+
+# ---- rescaling paths: scores that grow along the sequence ---------------------
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+@pytest.mark.parametrize("peak", [1.0, 3.0])
+def test_growing_and_peaked_scores(path, peak):
+    """Every query's RoPE part is a shared direction u and the RoPE key of token
+    t is 0.1 noise + (4 t / L) u, so scores rise by ~18 (natural units) along
+    the sequence: the running maximum keeps growing past the first tile's,
+    which forces the online-softmax rescale of the accumulator (lazy in the
+    absorb kernel).  Values keep unit scale.  peak scales u (a sharper
+    softmax)."""
+    d = synth.Dims(**LLAMA, s_q=2)
+    lens = [1500, 700]
+    inp = _wl(d, 2, lens, page=64, seed=21)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(5)
+    u = torch.randn(d.d_rope, generator=g, device=DEV) * peak
+    q = inp.q.float()
+    q[..., d.d_nope:] = u + 0.05 * torch.randn(q[..., d.d_nope:].shape, generator=g, device=DEV)
+    inp.q.copy_(q.to(inp.q.dtype))
+    for b, L in enumerate(lens):
+        nb = (L + 63) // 64
+        pages = inp.block_table[b, :nb].long()
+        rows = inp.latent[pages].reshape(nb * 64, -1).float()
+        t = torch.arange(nb * 64, device=DEV, dtype=torch.float32)[:, None]
+        rows[:, d.r:] = 0.1 * rows[:, d.r:] + (4.0 * t / L) * u[None, :] / peak
+        inp.latent[pages] = rows.to(inp.latent.dtype).reshape(nb, 64, -1)
+    out, lse = H.run_decode(inp, path, num_splits=1)
+    H.check_units(inp, out, lse, H.all_units(inp), "growing scores %s peak=%g" % (path, peak))
+    out2, lse2 = H.run_decode(inp, path)
+    H.check_units(inp, out2, lse2, H.all_units(inp), "growing scores %s peak=%g auto splits" % (path, peak))
