@@ -10,22 +10,23 @@
 // (query, head) rows at once: a dense contraction for the tensor cores.
 //
 // One CTA per (key-range split, sequence, block of 64 rows):
-//  * warp 0 loads the absorbed-query tile once (64 x 576, 72 KB) and streams
-//    64-token latent tiles (72 KB) with TMA into a 2-stage mbarrier ring;
-//  * warps 1 and 7 issue S = Q~ C^T as 36 tcgen05.mma (M=64, N=64, K=16),
-//    split along K into two double-buffered S halves in TMEM (one issuing
-//    thread cannot keep up with such small MMAs); warp 1 owns the 512 TMEM
-//    columns; warp 6 issues
-//    O += P C[:, :512] as 8 tcgen05.mma (M=64, N=256, K=16), reading the same
-//    latent tile as an MN-major B operand.  Two issuing threads keep the
-//    stage release (after PV) independent of the next tile's QK issue;
-//  * the M=64 accumulator uses 16 of every 32 TMEM lanes, so the two 256-wide
-//    halves of O sit interleaved at lane offsets 0 and 16 of the same 256
-//    columns; the S halves and buffers take columns 256..511;
-//  * warps 2-5 read S rows from TMEM, run the online softmax in the log2
-//    domain with lazy rescaling (O is only rescaled when a row max grows by
-//    more than 2^8), write P (bf16) to shared memory, and in the end scale O
-//    by 1/l and store the fp32 latent output and the log-sum-exp.
+//  * the absorbed-query tile (64 x 576) lives in TMEM and is the A operand of
+//    the score MMAs, so shared memory holds a 3-stage ring of 64-token latent
+//    tiles (72 KB each, TMA) next to the P tile;
+//  * TMEM: with M = 64 an accumulator occupies 16 of every 32 lanes.  Lanes
+//    0-15 of each quarter hold Q~ (columns 0..287, bf16 pairs) and the two S
+//    buffers (288..415); lanes 16-31 hold the two 256-column halves of O;
+//  * warp 1 owns the TMEM columns and issues S = Q~ C^T as 36 tcgen05.mma
+//    (M=64, N=64, K=16, A from TMEM); warp 6 issues O += P C[:, :512] as 8
+//    tcgen05.mma (M=64, N=256, A = P from shared memory, B = the same latent
+//    tile as an MN-major operand), so a stage is released as soon as its PV
+//    completes;
+//  * warps 2-5 load Q~ into TMEM, then per tile read S rows with tcgen05.ld,
+//    run the online softmax in the log2 domain with lazy rescaling (O is
+//    rescaled only when a row maximum grows by more than 2^8, through the
+//    16-lane TMEM shape so the Q~/S lanes are never touched), write P (bf16)
+//    to shared memory, and at the end stage O through shared memory to write
+//    the fp32 latent output and the log-sum-exp of the split.
 #include <math.h>
 
 #include "ptx.cuh"
@@ -42,23 +43,29 @@ constexpr int kDr = 64;
 constexpr int kE = kR + kDr;                 // 576 latent row elements
 constexpr int kM = 64;                       // (query, head) rows per CTA
 constexpr int kTk = 64;                      // tokens per tile
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kChunks = kE / 64;             // 128-byte column chunks of a row
-constexpr int kQChunk = kM * 128;
 constexpr int kKVChunk = kTk * 128;
-constexpr int kQBytes = kChunks * kQChunk;           // 73728
-constexpr int kStageBytes = kChunks * kKVChunk;      // 36864
+constexpr int kStageBytes = kChunks * kKVChunk;      // 73728
 constexpr int kPBytes = kM * 128;                    // 64 rows x 64 tokens (bf16)
-constexpr size_t kSmemBytes = (size_t)kQBytes + (size_t)kStages * kStageBytes + kPBytes + 1024;
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + kPBytes + 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol = 256;                  // S buffers: [half a|b][buffer 0|1] x kTk columns
-constexpr int kQkSplit = 18;                     // k-steps (of 36) issued by the first QK warp
-constexpr int kThreads = 8 * 32;
+constexpr uint32_t kQCols = kE / 2;                  // 288 columns of bf16 pairs
+constexpr uint32_t kSCol = kQCols;                   // S buffers at 288 and 352
+constexpr uint32_t kOLane = 16u << 16;               // O in lanes 16-31 of each quarter
+constexpr int kOStride = kR + 4;                     // staging pitch (floats) for the output
+constexpr int kThreads = 7 * 32;
 constexpr float kRescaleLog2 = 8.f;
+
+static_assert(kSCol + 2 * kTk <= kTmemCols, "Q~ and the S buffers must fit the low half-lanes");
+static_assert((size_t)kM * kOStride * 4 <= (size_t)kStages * kStageBytes, "output staging fits the ring");
 
 struct AbsorbParams {
   KvLayout ly;
   SplitPlan plan;
+  const __nv_bfloat16* qt;  // absorbed queries [rows, 512]
+  const __nv_bfloat16* q;   // queries [rows, d_nope + 64] (for q_rope)
+  int d_nope;
   float* o_part;   // [S, rows, 512] normalised latent outputs of each split
   float* lse;      // [S, rows] their log-sum-exp
   int s_q;
@@ -70,14 +77,12 @@ struct AbsorbParams {
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    absorb_decode_kernel(const __grid_constant__ CUtensorMap qt_map, const __grid_constant__ CUtensorMap qr_map,
-                         const __grid_constant__ CUtensorMap kv_map, const AbsorbParams p, int d_nope) {
+    absorb_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const AbsorbParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;
-  uint8_t* sKV = smem + kQBytes;
+  uint8_t* sKV = smem;
   uint8_t* sP = sKV + kStages * kStageBytes;
-  __shared__ __align__(8) uint64_t q_full, p_full, pv_done, qk_drain[2], pv_drain;
+  __shared__ __align__(8) uint64_t q_full, p_full, pv_done, qk_drain, pv_drain;
   __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -87,18 +92,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = blockIdx.y / p.hblocks, hb = blockIdx.y % p.hblocks;
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(&q_full, 1);
+    ptx::mbar_init(&q_full, 4);
     ptx::mbar_init(&p_full, 4);
     ptx::mbar_init(&pv_done, 1);
-    ptx::mbar_init(&qk_drain[0], 1);
-    ptx::mbar_init(&qk_drain[1], 1);
+    ptx::mbar_init(&qk_drain, 1);
     ptx::mbar_init(&pv_drain, 1);
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(&kv_full[s], 1);
       ptx::mbar_init(&kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(&s_full[s], 2);   // one commit from each QK issuer
+      ptx::mbar_init(&s_full[s], 1);
       ptx::mbar_init(&s_free[s], 4);
     }
     abort_flag = 0;
@@ -121,12 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
     if (lane == 0 && n_tiles > 0) {
-      ptx::prefetch_tmap(&qt_map);
-      ptx::prefetch_tmap(&qr_map);
       ptx::prefetch_tmap(&kv_map);
-      ptx::mbar_arrive_expect_tx(&q_full, kQBytes);
-      for (int c = 0; c < kR / 64; ++c) ptx::tma_load_2d(sQ + c * kQChunk, &qt_map, &q_full, 64 * c, (int)grow0);
-      ptx::tma_load_2d(sQ + (kR / 64) * kQChunk, &qr_map, &q_full, d_nope, (int)grow0);
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kStages, k = j / kStages;
@@ -143,35 +142,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = j + 1;
       }
       // no copy may still be landing in shared memory when the CTA retires
-      ptx::mbar_wait(&q_full, 0);
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
         ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1);
     }
-  } else if (warp == 1 || warp == 7) {
-    // ------------------------------------------------------- QK issuers
-    // One tcgen05.mma costs its issuing thread about as much time as a small
-    // (N=64) MMA takes to run, so two warps issue the 36 QK k-steps: warp 1
-    // k-steps [0, kQkSplit) into S half a, warp 7 the rest into S half b; the
-    // softmax adds the halves.  Warp 1 also owns the TMEM allocation.
-    const int half_q = warp == 7 ? 1 : 0;
+  } else if (warp == 1) {
+    // ---------------------------------------------- QK issuer, TMEM owner
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = ptx::idesc_bf16(kM, kTk, false, false);
-      const uint32_t q_addr = ptx::smem_u32(sQ), kv_addr = ptx::smem_u32(sKV);
-      const int k_lo = half_q ? kQkSplit : 0, k_hi = half_q ? kE / 16 : kQkSplit;
+      const uint32_t kv_addr = ptx::smem_u32(sKV);
       bool ok = ptx::mbar_wait(&q_full, 0);
+      ptx::tc_fence_after();
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kStages, sb = j & 1;
         ok = ptx::mbar_wait(&kv_full[s], (j / kStages) & 1);
         if (ok && j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t d = tmem + kSCol + (uint32_t)kTk * (2 * half_q + sb);
+        const uint32_t d = tmem + kSCol + (uint32_t)kTk * sb;
         const uint32_t st_addr = kv_addr + s * kStageBytes;
-        for (int kk = k_lo; kk < k_hi; ++kk) {
+#pragma unroll
+        for (int kk = 0; kk < kE / 16; ++kk) {
           const uint32_t koff = (kk >> 2), kin = (kk & 3) * 32;
-          const uint64_t a = ptx::umma_desc_sw128(q_addr + koff * kQChunk + kin, 16, 1024);
           const uint64_t bd = ptx::umma_desc_sw128(st_addr + koff * kKVChunk + kin, 16, 1024);
-          ptx::umma_bf16(d, a, bd, idesc_qk, kk > k_lo);
+          ptx::umma_bf16_ts(d, tmem + 8u * kk, bd, idesc_qk, kk > 0);
         }
         ptx::umma_commit(&s_full[sb]);
       }
@@ -180,13 +173,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicExch(&abort_flag, 1);
       }
       // every issued MMA has finished before TMEM is released
-      ptx::umma_commit(&qk_drain[half_q]);
-      ptx::mbar_wait(&qk_drain[half_q], 0);
+      ptx::umma_commit(&qk_drain);
+      ptx::mbar_wait(&qk_drain, 0);
     }
   } else if (warp == 6) {
     // ---------------------------------------------------------- PV issuer
-    // A second issuing thread: PV(j) goes out as soon as P(j) is ready, so
-    // the stage it releases is not held behind the next tile's QK.
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_pv = ptx::idesc_bf16(kM, 256, false, true);
       const uint32_t kv_addr = ptx::smem_u32(sKV), p_addr = ptx::smem_u32(sP);
@@ -203,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kTk / 16; ++kk) {
             const uint64_t a = ptx::umma_desc_sw128(p_addr + kk * 32, 16, 1024);
             const uint64_t bd = ptx::umma_desc_sw128(st_addr + (4 * h) * kKVChunk + kk * 16 * 128, kKVChunk, 1024);
-            ptx::umma_bf16(tmem + (h ? (16u << 16) : 0u), a, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            ptx::umma_bf16(tmem + kOLane + 256u * h, a, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
           }
         }
         ptx::umma_commit(&pv_done);
@@ -219,13 +210,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------- softmax + epilogue warps
     const int qd = warp & 3;                    // TMEM lane quarter of this warp
-    const int row = 16 * qd + (lane & 15);      // M-row (query, head) index
-    const int half = lane >> 4;                 // 0: O columns 0..255, 1: 256..511
+    const int row = 16 * qd + (lane & 15);      // S row held by lanes 0-15
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     const int r_local = hb * kM + row;
     const bool in_range = r_local < p.rows_unit;   // rows past the sequence's heads are padding
     const bool valid = in_range && L >= 0;
     const int vis = valid ? L - p.s_q + r_local / (p.rows_unit / p.s_q) + 1 : 0;
+    // lanes 16-31 address O through the 16-lane shape: this thread's O row
+    const int o_dp = 8 * (lane & 1) + (lane >> 2);
+
+    // Q~ = [q~ (512) ; q_rope (64)] of this row into TMEM (lanes 0-15), as
+    // bf16 pairs; lanes 16-31 store zeros into the O half-lanes, which the
+    // first PV overwrites.
+    {
+      const bool load = lane < 16 && in_range && grow0 + row < p.rows;
+      const long long grow = grow0 + row;
+      for (int c = 0; c < (int)kQCols / 32; ++c) {
+        uint32_t v[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const int col = 32 * c + e;            // bf16-pair column = element pair
+          uint4 w = make_uint4(0, 0, 0, 0);
+          if (load) {
+            if (col < kR / 2) w = *reinterpret_cast<const uint4*>(p.qt + grow * kR + 2 * col);
+            else w = *reinterpret_cast<const uint4*>(p.q + grow * (p.d_nope + kDr) + p.d_nope + 2 * (col - kR / 2));
+          }
+          v[e] = w.x;
+          v[e + 1] = w.y;
+          v[e + 2] = w.z;
+          v[e + 3] = w.w;
+        }
+        ptx::tmem_st32(tl + 32u * c, v);
+      }
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&q_full);
+    }
+
     float m_used = -INFINITY, l_sum = 0.f;
     bool ok = true;
     // After a failed (bounded) wait the warp stops waiting and only keeps the
@@ -238,31 +260,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sv[kTk];
       if (ok) {
         ptx::tc_fence_after();
-        uint32_t sb2[32];
         ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * sb, sv);
         ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * sb + 32u, sv + 32);
-        ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * (2 + sb), sb2);
         ptx::tmem_ld_wait();
-#pragma unroll
-        for (int t = 0; t < 32; ++t) sv[t] = __float_as_uint(__uint_as_float(sv[t]) + __uint_as_float(sb2[t]));
-        ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * (2 + sb) + 32u, sb2);
-        ptx::tmem_ld_wait();
-#pragma unroll
-        for (int t = 0; t < 32; ++t)
-          sv[32 + t] = __float_as_uint(__uint_as_float(sv[32 + t]) + __uint_as_float(sb2[t]));
       }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&s_free[sb]);
-      float pv[kTk];
       float factor = 1.f;
       int need = 0;
-      if (half == 0 && ok) {
+      if (lane < 16 && ok) {
         float mx = -INFINITY;
 #pragma unroll
         for (int t = 0; t < kTk; ++t) {
           const float x = (t0 + t < vis) ? __uint_as_float(sv[t]) * p.scale_log2 : -INFINITY;
-          pv[t] = x;
+          sv[t] = __float_as_uint(x);
           mx = fmaxf(mx, x);
         }
         if (m_used == -INFINITY) {
@@ -276,29 +288,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         float acc = 0.f;
 #pragma unroll
         for (int t = 0; t < kTk; ++t) {
-          const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(pv[t] - m_used);
-          pv[t] = e;
+          const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(__uint_as_float(sv[t]) - m_used);
+          sv[t] = __float_as_uint(e);
           acc += e;
         }
         l_sum += acc;
       } else {
 #pragma unroll
-        for (int t = 0; t < kTk; ++t) pv[t] = 0.f;
+        for (int t = 0; t < kTk; ++t) sv[t] = 0u;
       }
-      const float f_row = __shfl_sync(0xffffffffu, factor, lane & 15);
+      const float f_row = __shfl_sync(0xffffffffu, factor, o_dp);
       const bool any_rescale = __any_sync(0xffffffffu, need) != 0;
       // PV(j-1) must be done before O is rescaled and before P is overwritten
       if (ok && j >= 1) ok = ptx::mbar_wait(&pv_done, (j - 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (ok && any_rescale) {
         ptx::tc_fence_after();
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < kR / 64; ++c) {
           uint32_t ov[32];
-          ptx::tmem_ld32(tl + 32u * c, ov);
+          ptx::tmem_ld16x64(tl + kOLane + 64u * c, ov);
           ptx::tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f_row);
-          ptx::tmem_st32(tl + 32u * c, ov);
+          ptx::tmem_st16x64(tl + kOLane + 64u * c, ov);
         }
         ptx::tmem_st_wait();
       }
@@ -312,14 +324,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_uint4(0, 0, 0, 0);
         }
       }
-      if (half == 0) {
+      if (lane < 16) {
 #pragma unroll
         for (int g8 = 0; g8 < kTk / 8; ++g8) {
           uint4 v;
-          v.x = ptx::pack_bf16(pv[8 * g8 + 0], pv[8 * g8 + 1]);
-          v.y = ptx::pack_bf16(pv[8 * g8 + 2], pv[8 * g8 + 3]);
-          v.z = ptx::pack_bf16(pv[8 * g8 + 4], pv[8 * g8 + 5]);
-          v.w = ptx::pack_bf16(pv[8 * g8 + 6], pv[8 * g8 + 7]);
+          v.x = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 0]), __uint_as_float(sv[8 * g8 + 1]));
+          v.y = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 2]), __uint_as_float(sv[8 * g8 + 3]));
+          v.z = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 4]), __uint_as_float(sv[8 * g8 + 5]));
+          v.w = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 6]), __uint_as_float(sv[8 * g8 + 7]));
           *reinterpret_cast<uint4*>(sP + ptx::swz128(row, g8)) = v;
         }
       }
@@ -335,33 +347,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ----------------------------------------------------------- epilogue
     bool have_o = ok && n_tiles > 0 && ptx::mbar_wait(&pv_done, (n_tiles - 1) & 1);
     have_o = __all_sync(0xffffffffu, have_o);
-    ptx::tc_fence_after();
-    const float l_tot = __shfl_sync(0xffffffffu, l_sum, lane & 15);
-    const float m_tot = __shfl_sync(0xffffffffu, m_used, lane & 15);
-    const bool empty = !(l_tot > 0.f) || !have_o;
-    const float inv = empty ? 0.f : 1.f / l_tot;
-    const long long grow = grow0 + row;
-    float* dst = nullptr;
-    if (in_range && ok) dst = p.o_part + ((long long)split * p.rows + grow) * kR + half * 256;
-    for (int c = 0; c < 8; ++c) {
-      uint32_t ov[32];
-      if (have_o) {
-        ptx::tmem_ld32(tl + 32u * c, ov);
+    // the whole ring is idle now (every load was consumed): stage O there
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    float* stage = reinterpret_cast<float*>(sKV);
+    const float l_o = __shfl_sync(0xffffffffu, l_sum, o_dp);
+    const float inv_o = (l_o > 0.f && have_o) ? 1.f / l_o : 0.f;
+    if (have_o) {
+      ptx::tc_fence_after();
+      const int orow = 16 * qd + o_dp, par = (lane >> 1) & 1;
+      for (int c = 0; c < kR / 64; ++c) {
+        uint32_t ov[32];
+        ptx::tmem_ld16x64(tl + kOLane + 64u * c, ov);
         ptx::tmem_ld_wait();
-      }
-      if (dst) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          float4 v = empty ? make_float4(0.f, 0.f, 0.f, 0.f)
-                           : make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
-                                         __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
-          *reinterpret_cast<float4*>(dst + 32 * c + e) = v;
-        }
+        for (int e = 0; e < 32; ++e) stage[orow * kOStride + 64 * c + par + 2 * e] = __uint_as_float(ov[e]) * inv_o;
       }
     }
-    if (in_range && ok && half == 0) {
-      const float lse = empty ? -INFINITY : (m_tot + log2f(l_tot)) * 0.69314718055994531f;
-      p.lse[(long long)split * p.rows + grow] = lse;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int tid = threadIdx.x - 64;
+    for (int idx = tid; idx < kM * (kR / 4); idx += 128) {
+      const int rr = idx / (kR / 4), c4 = (idx % (kR / 4)) * 4;
+      if (hb * kM + rr >= p.rows_unit || !ok) continue;
+      const long long grow = grow0 + rr;
+      float4 v = have_o ? *reinterpret_cast<const float4*>(stage + rr * kOStride + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(p.o_part + ((long long)split * p.rows + grow) * kR + c4) = v;
+    }
+    if (in_range && ok && lane < 16) {
+      const bool empty = !(l_sum > 0.f) || !have_o;
+      const float lse = empty ? -INFINITY : (m_used + log2f(l_sum)) * 0.69314718055994531f;
+      p.lse[(long long)split * p.rows + grow0 + row] = lse;
     }
   }
   // ------------------------------------------------------------ teardown
@@ -426,13 +440,14 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
   if (e != cudaSuccess) return e;
   long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
                                         : (long long)p.ly.num_pages * p.ly.page_size;
-  CUtensorMap qt_map, qr_map, kv_map;
-  if (!make_2d_map(&qt_map, w.qt, kR, p.rows, kR, kM) || !make_2d_map(&qr_map, q, p.d_qk, p.rows, p.d_qk, kM) ||
-      !make_2d_map(&kv_map, latent, kE, nrows, kE, kTk))
-    return cudaErrorInvalidValue;
+  CUtensorMap kv_map;
+  if (!make_2d_map(&kv_map, latent, kE, nrows, kE, kTk)) return cudaErrorInvalidValue;
   AbsorbParams prm;
   prm.ly = p.ly;
   prm.plan = p.plan;
+  prm.qt = (const __nv_bfloat16*)w.qt;
+  prm.q = (const __nv_bfloat16*)q;
+  prm.d_nope = d.d_nope;
   prm.o_part = w.o_part;
   prm.lse = w.lse_part;
   prm.s_q = d.s_q;
@@ -444,7 +459,7 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
   e = ensure_smem_limit((const void*)absorb_decode_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(S, p.ly.batch * prm.hblocks);
-  absorb_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(qt_map, qr_map, kv_map, prm, d.d_nope);
+  absorb_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(kv_map, prm);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
