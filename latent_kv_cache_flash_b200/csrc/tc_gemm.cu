@@ -158,20 +158,20 @@ __global__ void __launch_bounds__(256) combine_lat_kernel(int S, const float* __
 
 // ------------------------------------------------------------- up_proj
 // out[row] = o_lat[row] W_uv^g.  CTA: 16 rows of group g x 128 outputs,
-// 4 warps of 32 outputs; K = 512 in 64-wide chunks, double-buffered cp.async.
-constexpr int kUpRows = 16, kUpN = 128, kUpKC = 64;
-constexpr int kUpApitch = (kUpKC + 8) * 2;     // 144 B
+// 4 warps of 32 outputs; the whole K = 512 of both operands is fetched with
+// cp.async in one go (A 16 KB, B 128 KB), so the GEMM pays one load latency.
+constexpr int kUpRows = 16, kUpN = 128;
+constexpr int kUpApitch = (kLat + 8) * 2;      // 1040 B
 constexpr int kUpBpitch = (kUpN + 8) * 2;      // 272 B
 constexpr int kUpAbytes = kUpRows * kUpApitch;
-constexpr int kUpBbytes = kUpKC * kUpBpitch;
-constexpr size_t kUpSmem = 2 * (size_t)(kUpAbytes + kUpBbytes);
+constexpr int kUpBbytes = kLat * kUpBpitch;
+constexpr size_t kUpSmem = (size_t)kUpAbytes + kUpBbytes;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool pred) {
   const int sz = pred ? 16 : 0;
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict__ o_lat,
@@ -180,53 +180,38 @@ __global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict
   extern __shared__ __align__(16) uint8_t sm[];
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t base = ptx::smem_u32(sm);
+  const uint32_t a = ptx::smem_u32(sm), b = a + kUpAbytes;
   auto grow_of = [&](int rr) -> long long {
     const int lr = blockIdx.x * kUpRows + rr;
     return lr < rows_g ? (long long)(lr / m) * n_h + g * m + lr % m : -1;
   };
   const bf16* Wg = W_uv + (size_t)g * kLat * kUpN;
-  auto load_chunk = [&](int kc, int buf) {
-    const uint32_t a = base + buf * (kUpAbytes + kUpBbytes);
-    const uint32_t b = a + kUpAbytes;
-    for (int i = threadIdx.x; i < kUpRows * (kUpKC / 8); i += blockDim.x) {
-      const int rr = i / (kUpKC / 8), c = i % (kUpKC / 8);
-      const long long grow = grow_of(rr);
-      cp_async16(a + rr * kUpApitch + c * 16, o_lat + (grow < 0 ? 0 : grow) * kLat + kc + c * 8, grow >= 0);
-    }
-    for (int i = threadIdx.x; i < kUpKC * (kUpN / 8); i += blockDim.x) {
-      const int kk = i / (kUpN / 8), c = i % (kUpN / 8);
-      cp_async16(b + kk * kUpBpitch + c * 16, Wg + (size_t)(kc + kk) * kUpN + c * 8, true);
-    }
-    cp_async_commit();
-  };
+  for (int i = threadIdx.x; i < kUpRows * (kLat / 8); i += blockDim.x) {
+    const int rr = i / (kLat / 8), c = i % (kLat / 8);
+    const long long grow = grow_of(rr);
+    cp_async16(a + rr * kUpApitch + c * 16, o_lat + (grow < 0 ? 0 : grow) * kLat + c * 8, grow >= 0);
+  }
+  for (int i = threadIdx.x; i < kLat * (kUpN / 8); i += blockDim.x) {
+    const int kk = i / (kUpN / 8), c = i % (kUpN / 8);
+    cp_async16(b + kk * kUpBpitch + c * 16, Wg + (size_t)kk * kUpN + c * 8, true);
+  }
+  cp_async_commit();
+  cp_async_wait0();
+  __syncthreads();
   float acc[4][4];
 #pragma unroll
   for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-  load_chunk(0, 0);
-  for (int c = 0; c < kLat / kUpKC; ++c) {
-    if (c + 1 < kLat / kUpKC) {
-      load_chunk((c + 1) * kUpKC, (c + 1) & 1);
-      cp_async_wait1();
-    } else {
-      cp_async_wait0();
-    }
-    __syncthreads();
-    const uint32_t a = base + (c & 1) * (kUpAbytes + kUpBbytes);
-    const uint32_t b = a + kUpAbytes;
+#pragma unroll 4
+  for (int k0 = 0; k0 < kLat; k0 += 16) {
+    uint32_t af[4];
+    ldsm_a(a, kUpApitch, 0, k0, af);
 #pragma unroll
-    for (int k0 = 0; k0 < kUpKC; k0 += 16) {
-      uint32_t af[4];
-      ldsm_a(a, kUpApitch, 0, k0, af);
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        uint32_t bf[4];
-        ldsm_b_kn(b, kUpBpitch, warp * 32 + np * 16, k0, bf);
-        ptx::mma_bf16_16816(acc[2 * np], af, bf[0], bf[1]);
-        ptx::mma_bf16_16816(acc[2 * np + 1], af, bf[2], bf[3]);
-      }
+    for (int np = 0; np < 2; ++np) {
+      uint32_t bf[4];
+      ldsm_b_kn(b, kUpBpitch, warp * 32 + np * 16, k0, bf);
+      ptx::mma_bf16_16816(acc[2 * np], af, bf[0], bf[1]);
+      ptx::mma_bf16_16816(acc[2 * np + 1], af, bf[2], bf[3]);
     }
-    __syncthreads();
   }
   const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
