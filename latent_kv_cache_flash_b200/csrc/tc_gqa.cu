@@ -268,31 +268,49 @@ __global__ void __launch_bounds__(kThreads, 2)
     ml[kConsumerWarps * 16 + warp * 16 + gid + 8] = lrow[1];
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-  // each warp finishes 16 / ts rows of its row block
-  const int rows_per = 16 / ts;
-  for (int rr = slice * rows_per; rr < (slice + 1) * rows_per; ++rr) {
-    const int r = (rb0 + rbl) * 16 + rr;
-    if (r >= p.rows_unit) break;
+  // Merge: every consumer thread takes (row, 4 columns) pieces of the
+  // CTA's rows; the ts partial states of a row are combined with per-row
+  // weights held in registers.
+  const int tid = threadIdx.x;
+  for (int idx = tid; idx < p.rbc * 16 * (kDv / 4); idx += kConsumerWarps * 32) {
+    const int rl = idx / (kDv / 4), d4 = (idx % (kDv / 4)) * 4;
+    const int rbl2 = rl >> 4, rr = rl & 15;
+    const int r = (rb0 + rbl2) * 16 + rr;
+    if (r >= p.rows_unit) continue;
     const int i = r / p.m, h = g * p.m + r % p.m;
     const long long gr = ((long long)b * p.s_q + i) * p.n_h + h;
     float mt = -INFINITY;
-    for (int w = 0; w < ts; ++w) mt = fmaxf(mt, ml[(rbl * ts + w) * 16 + rr]);
-    float wsum = 0.f, wgt[kConsumerWarps];
-    for (int w = 0; w < ts; ++w) {
-      const float mw = ml[(rbl * ts + w) * 16 + rr];
-      wgt[w] = mw == -INFINITY ? 0.f : ptx::fast_exp2(mw - mt);
-      wsum += wgt[w] * ml[kConsumerWarps * 16 + (rbl * ts + w) * 16 + rr];
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w)
+      if (w < ts) mt = fmaxf(mt, ml[(rbl2 * ts + w) * 16 + rr]);
+    float wsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      if (w < ts) {
+        const float mwv = ml[(rbl2 * ts + w) * 16 + rr];
+        const float wv = mwv == -INFINITY ? 0.f : ptx::fast_exp2(mwv - mt);
+        wsum += wv * ml[kConsumerWarps * 16 + (rbl2 * ts + w) * 16 + rr];
+        const float4 o4 = *reinterpret_cast<const float4*>(&ob[((rbl2 * ts + w) * 16 + rr) * kOStride + d4]);
+        acc.x = fmaf(wv, o4.x, acc.x);
+        acc.y = fmaf(wv, o4.y, acc.y);
+        acc.z = fmaf(wv, o4.z, acc.z);
+        acc.w = fmaf(wv, o4.w, acc.w);
+      }
     }
     const bool empty = !(wsum > 0.f);
     const float inv = empty ? 0.f : 1.f / wsum;
-    for (int d = lane; d < kDv; d += 32) {
-      float acc = 0.f;
-      for (int w = 0; w < ts; ++w) acc += wgt[w] * ob[((rbl * ts + w) * 16 + rr) * kOStride + d];
-      acc *= inv;
-      if (p.o_part) p.o_part[((long long)split * p.rows + gr) * kDv + d] = acc;
-      else p.out[gr * kDv + d] = __float2bfloat16_rn(acc);
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
+    if (p.o_part) {
+      *reinterpret_cast<float4*>(p.o_part + ((long long)split * p.rows + gr) * kDv + d4) = acc;
+    } else {
+      *reinterpret_cast<uint2*>(p.out + gr * kDv + d4) =
+          make_uint2(ptx::pack_bf16(acc.x, acc.y), ptx::pack_bf16(acc.z, acc.w));
     }
-    if (lane == 0 && p.lse) {
+    if (d4 == 0 && p.lse) {
       const float lse = empty ? -INFINITY : (mt + log2f(wsum)) * 0.69314718055994531f;
       p.lse[p.o_part ? (long long)split * p.rows + gr : gr] = lse;
     }
