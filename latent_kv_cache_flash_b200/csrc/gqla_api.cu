@@ -80,6 +80,12 @@ SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, 
     slots = (long long)num_sms() * 1;
     unit_bytes = 2.0 * (d.r + d.d_rope);
     part_bytes = (double)rows * (d.r + 1) * 4 * 2;
+  } else if ((d.n_h / d.G) * d.s_q >= 64 && tc) {
+    // the tcgen05 GQA kernel: 128-row blocks, one CTA per SM
+    units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 127) / 128);
+    slots = (long long)num_sms();
+    unit_bytes = 2.0 * (d.d_nope + d.d_rope + d.d_v);
+    part_bytes = (double)rows * (d.d_v + 1) * 4 * 2;
   } else {
     units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 63) / 64);
     slots = (long long)num_sms() * 2;

@@ -11,6 +11,12 @@ bool tc_gqa_supports(const Problem& p);
 cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
                           float* o_part, float* lse_dst, int32_t* st, cudaStream_t s);
 
+// GQA decode for m * s_q >= 64 rows per group: tcgen05/TMEM (tc_gqa_wide.cu);
+// tc_gqa_decode hands such problems to it.
+bool tc_gqa_wide_supports(const Problem& p);
+cudaError_t tc_gqa_wide_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
+                               float* o_part, float* lse_dst, int32_t* st, cudaStream_t s);
+
 // MQA-absorb decode: absorbed query, latent attention on tcgen05/TMEM, combine,
 // up-projection.
 bool tc_absorb_supports(const Problem& p);

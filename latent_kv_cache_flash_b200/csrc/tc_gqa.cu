@@ -360,6 +360,7 @@ bool tc_gqa_supports(const Problem& p) {
 
 cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
                           float* o_part, float* lse_dst, int32_t* st, cudaStream_t s) {
+  if (tc_gqa_wide_supports(p)) return tc_gqa_wide_decode(p, q, k_pool, v_pool, out, o_part, lse_dst, st, s);
   const auto& d = p.d;
   long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
                                         : (long long)p.ly.num_pages * p.ly.page_size;

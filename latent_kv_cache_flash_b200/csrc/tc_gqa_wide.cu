@@ -1,0 +1,426 @@
+// GQA-path decode for many rows per group (m * s_q >= 64), bf16, on tcgen05.
+//
+// Grouped-query decode over the per-group expanded cache ("GQLA" chatpaper.ai
+// Abstract: a GQA path with a per-group expanded cache; "Grouped Query
+// Attention (GQA)" glossary, "Fonctionnement de la GQA").  With few groups
+// and several new tokens per sequence a group serves hundreds of (query,
+// head) rows, and the contraction becomes tensor-bound: this kernel runs it
+// on the 5th-generation tensor cores with the rows as the MMA's M.
+//
+// One CTA per (key-range split, sequence, group, block of 128 rows):
+//  * the 128 x 192 query tile is gathered into 128-byte-swizzled shared
+//    memory once; 64-token K (64 x 192) and V (64 x 128) tiles stream in with
+//    TMA (3-D views of the pools) into a 4-stage mbarrier ring;
+//  * warp 1 issues S = Q K^T (12 tcgen05.mma, M=128, N=64, K=16) into a
+//    double-buffered S in TMEM; warp 6 issues O += P V (4 tcgen05.mma,
+//    M=128, N=128, K=16, V as an MN-major operand) into O in TMEM;
+//  * warps 2-5 own one row each: online softmax in the log2 domain with lazy
+//    rescaling of O (only when a row maximum grows by more than 2^8), P to
+//    shared memory, and the normalised output and log-sum-exp at the end.
+#include <math.h>
+
+#include "ptx.cuh"
+#include "tc.h"
+
+namespace gqla {
+
+namespace {
+
+constexpr int kDqk = 192;
+constexpr int kDv = 128;
+constexpr int kM = 128;                       // (query, head) rows per CTA
+constexpr int kT = 64;                        // tokens per tile
+constexpr int kStages = 4;
+constexpr int kKChunks = kDqk / 64;           // 3 K chunks of 64 dims
+constexpr int kVChunks = kDv / 64;            // 2 V chunks
+constexpr int kChunkBytes = kT * 128;         // 8 KB
+constexpr int kStageBytes = (kKChunks + kVChunks) * kChunkBytes;   // 40 KB
+constexpr int kQChunkBytes = kM * 128;        // 16 KB
+constexpr int kQBytes = kKChunks * kQChunkBytes;                     // 48 KB
+constexpr int kPBytes = kM * 128;             // 128 rows x 64 tokens (bf16)
+constexpr size_t kSmemBytes = (size_t)kQBytes + (size_t)kStages * kStageBytes + kPBytes + 1024;
+constexpr uint32_t kTmemCols = 256;           // S: 2 x 64, O: 128
+constexpr uint32_t kSCol = 0, kOCol = 128;
+constexpr int kThreads = 7 * 32;
+constexpr float kRescaleLog2 = 8.f;
+
+struct WideParams {
+  KvLayout ly;
+  SplitPlan plan;
+  const __nv_bfloat16* q;
+  __nv_bfloat16* out;
+  float* o_part;
+  float* lse;
+  int n_h, G, m, s_q;
+  int rows_unit;      // m * s_q
+  int rblocks;        // ceil(rows_unit / 128)
+  float scale_log2;
+  long long rows;     // B * s_q * n_h
+  int32_t* st;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gqa_wide_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                    const WideParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + kQBytes;
+  uint8_t* sP = sKV + kStages * kStageBytes;
+  __shared__ __align__(8) uint64_t q_full, p_full, pv_done, qk_drain, pv_drain;
+  __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x;
+  const int b = blockIdx.y / p.G, g = blockIdx.y % p.G;
+  const int rb = blockIdx.z;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&q_full, 4);
+    ptx::mbar_init(&p_full, 4);
+    ptx::mbar_init(&pv_done, 1);
+    ptx::mbar_init(&qk_drain, 1);
+    ptx::mbar_init(&pv_drain, 1);
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(&kv_full[s], 1);
+      ptx::mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&s_full[s], 1);
+      ptx::mbar_init(&s_free[s], 4);
+    }
+    abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&tmem_base_sh, kTmemCols);
+    ptx::tmem_relinquish();
+    ptx::tc_fence_before();
+  }
+  int L = seq_len_checked(p.ly, b, p.s_q, (split == 0 && g == 0 && rb == 0) ? p.st : nullptr);
+  if (!seq_pages_ok(p.ly, b, L, p.st)) L = -1;   // includes a __syncthreads
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int t_begin = split * p.plan.chunk;
+  const int t_stop = L < 0 ? t_begin : min(t_begin + p.plan.chunk, L);
+  const int n_tiles = t_stop > t_begin ? (t_stop - t_begin + kT - 1) / kT : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0 && n_tiles > 0) {
+      ptx::prefetch_tmap(&kmap);
+      ptx::prefetch_tmap(&vmap);
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % kStages, k = j / kStages;
+        if (k > 0 && !ptx::mbar_wait(&kv_empty[s], (k - 1) & 1)) {
+          flag_status(p.st, GQLA_DEV_TIMEOUT);
+          atomicExch(&abort_flag, 1);
+          break;
+        }
+        if (*(volatile int*)&abort_flag) break;
+        const int row0 = (int)token_row(p.ly, b, t_begin + j * kT, nullptr);
+        uint8_t* dst = sKV + s * kStageBytes;
+        ptx::mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
+        for (int c = 0; c < kKChunks; ++c)
+          ptx::tma_load_3d(dst + c * kChunkBytes, &kmap, &kv_full[s], 64 * c, g, row0);
+        for (int c = 0; c < kVChunks; ++c)
+          ptx::tma_load_3d(dst + (kKChunks + c) * kChunkBytes, &vmap, &kv_full[s], 64 * c, g, row0);
+        issued = j + 1;
+      }
+      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+        ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------- QK issuer, TMEM owner
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t idesc_qk = ptx::idesc_bf16(kM, kT, false, false);
+      const uint32_t q_addr = ptx::smem_u32(sQ), kv_addr = ptx::smem_u32(sKV);
+      bool ok = ptx::mbar_wait(&q_full, 0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kStages, sb = j & 1;
+        ok = ptx::mbar_wait(&kv_full[s], (j / kStages) & 1);
+        if (ok && j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint32_t st_addr = kv_addr + s * kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < kDqk / 16; ++kk) {
+          const uint32_t koff = kk >> 2, kin = (kk & 3) * 32;
+          const uint64_t a = ptx::umma_desc_sw128(q_addr + koff * kQChunkBytes + kin, 16, 1024);
+          const uint64_t bd = ptx::umma_desc_sw128(st_addr + koff * kChunkBytes + kin, 16, 1024);
+          ptx::umma_bf16(tmem + kSCol + (uint32_t)kT * sb, a, bd, idesc_qk, kk > 0);
+        }
+        ptx::umma_commit(&s_full[sb]);
+      }
+      if (!ok) {
+        flag_status(p.st, GQLA_DEV_TIMEOUT);
+        atomicExch(&abort_flag, 1);
+      }
+      ptx::umma_commit(&qk_drain);
+      ptx::mbar_wait(&qk_drain, 0);
+    }
+  } else if (warp == 6) {
+    // ---------------------------------------------------------- PV issuer
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t idesc_pv = ptx::idesc_bf16(kM, kDv, false, true);
+      const uint32_t kv_addr = ptx::smem_u32(sKV), p_addr = ptx::smem_u32(sP);
+      bool ok = true;
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kStages;
+        ok = ptx::mbar_wait(&p_full, j & 1);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint32_t v_addr = kv_addr + s * kStageBytes + kKChunks * kChunkBytes;
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk) {
+          const uint64_t a = ptx::umma_desc_sw128(p_addr + kk * 32, 16, 1024);
+          const uint64_t bd = ptx::umma_desc_sw128(v_addr + kk * 16 * 128, kChunkBytes, 1024);
+          ptx::umma_bf16(tmem + kOCol, a, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::umma_commit(&pv_done);
+        ptx::umma_commit(&kv_empty[s]);
+      }
+      if (!ok) {
+        flag_status(p.st, GQLA_DEV_TIMEOUT);
+        atomicExch(&abort_flag, 1);
+      }
+      ptx::umma_commit(&pv_drain);
+      ptx::mbar_wait(&pv_drain, 0);
+    }
+  } else {
+    // ------------------------------------------- softmax + epilogue warps
+    const int qd = warp & 3;
+    const int row = 32 * qd + lane;             // M row = TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+    const int r_local = rb * kM + row;
+    const bool in_range = r_local < p.rows_unit;
+    const bool valid = in_range && L >= 0;
+    const int i_q = in_range ? r_local / p.m : 0;
+    const long long grow = in_range ? ((long long)b * p.s_q + i_q) * p.n_h + g * p.m + r_local % p.m : 0;
+    const int vis = valid ? L - p.s_q + i_q + 1 : 0;
+    // this row's query into the swizzled Q tile (zeros for padding rows)
+    for (int c = 0; c < kKChunks; ++c) {
+#pragma unroll
+      for (int gi = 0; gi < 8; ++gi) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (in_range) v = *reinterpret_cast<const uint4*>(p.q + grow * kDqk + 64 * c + 8 * gi);
+        *reinterpret_cast<uint4*>(sQ + c * kQChunkBytes + ptx::swz128(row, gi)) = v;
+      }
+    }
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&q_full);
+
+    float m_used = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int sb = j & 1, s = j % kStages;
+      const int t0 = t_begin + j * kT;
+      if (ok) ok = ptx::mbar_wait(&s_full[sb], (j >> 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      uint32_t sv[kT];
+      if (ok) {
+        ptx::tc_fence_after();
+        ptx::tmem_ld32(tl + kSCol + (uint32_t)kT * sb, sv);
+        ptx::tmem_ld32(tl + kSCol + (uint32_t)kT * sb + 32u, sv + 32);
+        ptx::tmem_ld_wait();
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s_free[sb]);
+      float factor = 1.f;
+      int need = 0;
+      if (ok) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < kT; ++t) {
+          const float x = (t0 + t < vis) ? __uint_as_float(sv[t]) * p.scale_log2 : -INFINITY;
+          sv[t] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+        if (m_used == -INFINITY) {
+          m_used = mx;
+        } else if (mx > m_used + kRescaleLog2) {
+          factor = ptx::fast_exp2(m_used - mx);
+          need = 1;
+          l_sum *= factor;
+          m_used = mx;
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < kT; ++t) {
+          const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(__uint_as_float(sv[t]) - m_used);
+          sv[t] = __float_as_uint(e);
+          acc += e;
+        }
+        l_sum += acc;
+      } else {
+#pragma unroll
+        for (int t = 0; t < kT; ++t) sv[t] = 0u;
+      }
+      const bool any_rescale = __any_sync(0xffffffffu, need) != 0;
+      if (ok && j >= 1) ok = ptx::mbar_wait(&pv_done, (j - 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok && any_rescale) {
+        ptx::tc_fence_after();
+        for (int c = 0; c < kDv / 32; ++c) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(tl + kOCol + 32u * c, ov);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+          ptx::tmem_st32(tl + kOCol + 32u * c, ov);
+        }
+        ptx::tmem_st_wait();
+      }
+      if (t0 + kT > L) {
+        // value rows past the sequence may hold anything: zero them for PV
+        const int tid = threadIdx.x - 64;
+        for (int idx = tid; idx < kT * kVChunks * 8; idx += 128) {
+          const int tok = idx / (kVChunks * 8), rem = idx % (kVChunks * 8);
+          if (t0 + tok >= L)
+            *reinterpret_cast<uint4*>(sKV + s * kStageBytes + (kKChunks + rem / 8) * kChunkBytes +
+                                      ptx::swz128(tok, rem % 8)) = make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int g8 = 0; g8 < kT / 8; ++g8) {
+        uint4 v;
+        v.x = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 0]), __uint_as_float(sv[8 * g8 + 1]));
+        v.y = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 2]), __uint_as_float(sv[8 * g8 + 3]));
+        v.z = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 4]), __uint_as_float(sv[8 * g8 + 5]));
+        v.w = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 6]), __uint_as_float(sv[8 * g8 + 7]));
+        *reinterpret_cast<uint4*>(sP + ptx::swz128(row, g8)) = v;
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (lane == 0) ptx::mbar_arrive(&p_full);
+    }
+    if (!ok && lane == 0) {
+      flag_status(p.st, GQLA_DEV_TIMEOUT);
+      atomicExch(&abort_flag, 1);
+    }
+    // ----------------------------------------------------------- epilogue
+    bool have_o = ok && n_tiles > 0 && ptx::mbar_wait(&pv_done, (n_tiles - 1) & 1);
+    have_o = __all_sync(0xffffffffu, have_o);
+    ptx::tc_fence_after();
+    const bool empty = !(l_sum > 0.f) || !have_o;
+    const float inv = empty ? 0.f : 1.f / l_sum;
+    for (int c = 0; c < kDv / 32; ++c) {
+      uint32_t ov[32];
+      if (have_o) {
+        ptx::tmem_ld32(tl + kOCol + 32u * c, ov);
+        ptx::tmem_ld_wait();
+      }
+      if (in_range && ok) {
+        if (p.o_part) {
+          float* dst = p.o_part + ((long long)split * p.rows + grow) * kDv + 32 * c;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + e) =
+                empty ? make_float4(0.f, 0.f, 0.f, 0.f)
+                      : make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
+                                    __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
+        } else {
+          __nv_bfloat16* dst = p.out + grow * kDv + 32 * c;
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = ptx::pack_bf16(empty ? 0.f : __uint_as_float(ov[e]) * inv, empty ? 0.f : __uint_as_float(ov[e + 1]) * inv);
+            w.y = ptx::pack_bf16(empty ? 0.f : __uint_as_float(ov[e + 2]) * inv, empty ? 0.f : __uint_as_float(ov[e + 3]) * inv);
+            w.z = ptx::pack_bf16(empty ? 0.f : __uint_as_float(ov[e + 4]) * inv, empty ? 0.f : __uint_as_float(ov[e + 5]) * inv);
+            w.w = ptx::pack_bf16(empty ? 0.f : __uint_as_float(ov[e + 6]) * inv, empty ? 0.f : __uint_as_float(ov[e + 7]) * inv);
+            *reinterpret_cast<uint4*>(dst + e) = w;
+          }
+        }
+      }
+    }
+    if (in_range && ok && p.lse) {
+      const float lse = empty ? -INFINITY : (m_used + log2f(l_sum)) * 0.69314718055994531f;
+      p.lse[p.o_part ? (long long)split * p.rows + grow : grow] = lse;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)f;
+  }
+  return fn;
+}
+
+bool pool_map(CUtensorMap* map, const void* base, int dim, int G, long long nrows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3] = {(cuuint64_t)dim, (cuuint64_t)G, (cuuint64_t)nrows};
+  cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * 2 * G};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kT};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tc_gqa_wide_supports(const Problem& p) {
+  const auto& d = p.d;
+  if (d.dtype != GQLA_BF16 || p.d_qk != kDqk || d.d_v != kDv) return false;
+  if (p.m * d.s_q < 64) return false;
+  if (p.ly.page_size != 0 && p.ly.page_size % kT != 0) return false;
+  if ((long long)p.ly.batch * d.G > 65535) return false;
+  return true;
+}
+
+cudaError_t tc_gqa_wide_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
+                               float* o_part, float* lse_dst, int32_t* st, cudaStream_t s) {
+  const auto& d = p.d;
+  const long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
+                                              : (long long)p.ly.num_pages * p.ly.page_size;
+  CUtensorMap kmap, vmap;
+  if (!pool_map(&kmap, k_pool, kDqk, d.G, nrows) || !pool_map(&vmap, v_pool, kDv, d.G, nrows))
+    return cudaErrorInvalidValue;
+  WideParams prm;
+  prm.ly = p.ly;
+  prm.plan = p.plan;
+  prm.q = (const __nv_bfloat16*)q;
+  prm.out = (__nv_bfloat16*)out;
+  prm.o_part = o_part;
+  prm.lse = lse_dst;
+  prm.n_h = d.n_h;
+  prm.G = d.G;
+  prm.m = p.m;
+  prm.s_q = d.s_q;
+  prm.rows_unit = p.m * d.s_q;
+  prm.rblocks = (prm.rows_unit + kM - 1) / kM;
+  prm.scale_log2 = d.scale * 1.4426950408889634f;
+  prm.rows = p.rows;
+  prm.st = st;
+  cudaError_t e = ensure_smem_limit((const void*)gqa_wide_kernel, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.plan.num_splits, p.ly.batch * d.G, prm.rblocks);
+  gqa_wide_kernel<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace gqla

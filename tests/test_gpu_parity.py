@@ -270,3 +270,14 @@ def test_growing_and_peaked_scores(path, peak):
     H.check_units(inp, out, lse, H.all_units(inp), "growing scores %s peak=%g" % (path, peak))
     out2, lse2 = H.run_decode(inp, path)
     H.check_units(inp, out2, lse2, H.all_units(inp), "growing scores %s peak=%g auto splits" % (path, peak))
+
+
+@pytest.mark.parametrize("G,s_q", [(2, 2), (1, 2), (4, 4)])
+@pytest.mark.parametrize("splits", [0, 3])
+def test_gqa_many_rows_per_group_paged(G, s_q, splits):
+    """m * s_q >= 64 rows per group (the tensor-core GQA kernel), paged and
+    ragged, with and without split-KV."""
+    d = synth.Dims(n_h=128, G=G, d_nope=128, d_rope=64, d_v=128, r=512, s_q=s_q)
+    inp = _wl(d, 3, [777, 1500, 64], page=64, seed=40 + G)
+    out, lse = H.run_decode(inp, "gqa", num_splits=splits)
+    H.check_units(inp, out, lse, H.sample_units(inp, 5, seed=G), "gqa wide G=%d s_q=%d S=%d" % (G, s_q, splits))
