@@ -265,6 +265,14 @@ def run_ours(args):
 
     # the resident per-group cache of all tokens (a prefill-time cost, timed on its own)
     gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0, status)
+    # the step's new tokens [c_KV ; k_rope], resident on the device; each step
+    # writes them into the latent pool (they are the rows already there, so
+    # every step sees the same cache)
+    Lmax = wl.seq_len
+    new_rows = inp.latent[:, Lmax - d.s_q:Lmax].contiguous()
+
+    def append_latent():
+        gqla.gqla_append_tokens(dims, lay, new_rows, inp.latent, dev_status=status)
 
     def expand_tail():
         gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, d.s_q, status)
@@ -276,17 +284,20 @@ def run_ours(args):
         gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out_g, lse_g, 0, ws_g, status)
 
     def step():
+        append_latent()
         expand_tail()
         absorb()
         gqa()
 
-    # The two paths of a step share no data: the absorb path runs on a second
-    # stream, forked from and joined back into the main one, so its CTAs and
-    # the GQA path's share the machine.
+    # The two paths of a step share no data once the new rows are in the
+    # latent pool: the absorb path runs on a second stream, forked from and
+    # joined back into the main one, so its CTAs and the GQA path's share the
+    # machine.
     side = torch.cuda.Stream(dev)
 
     def step_overlapped():
         main = torch.cuda.current_stream(dev)   # the capture stream while a graph is recorded
+        append_latent()
         fork = torch.cuda.Event()
         fork.record(main)
         side.wait_event(fork)
@@ -342,6 +353,7 @@ def run_ours(args):
     ms_absorb = timed(absorb, reps) / reps
     ms_gqa = timed(gqa, reps) / reps
     ms_tail = timed(expand_tail, reps) / reps
+    ms_append = timed(append_latent, reps) / reps
     ms_expand_full = timed(lambda: gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0,
                                                           status), 3) / 3
 
@@ -349,13 +361,12 @@ def run_ours(args):
     # inputs (queries and the new tokens' latent rows) go host->device, both
     # paths' outputs come back device->host, inside the timed region
     q_host = inp.q.cpu().pin_memory()
-    Lmax = wl.seq_len
-    new_rows_host = inp.latent[:, Lmax - d.s_q:Lmax].cpu().pin_memory()
+    new_rows_host = new_rows.cpu().pin_memory()
     out_host = torch.empty((2,) + tuple(out_a.shape), dtype=out_a.dtype).pin_memory()
 
     def e2e_step():
         inp.q.copy_(q_host, non_blocking=True)
-        inp.latent[:, Lmax - d.s_q:Lmax].copy_(new_rows_host, non_blocking=True)
+        new_rows.copy_(new_rows_host, non_blocking=True)
         step()
         out_host[0].copy_(out_a, non_blocking=True)
         out_host[1].copy_(out_g, non_blocking=True)
@@ -410,7 +421,8 @@ def run_ours(args):
         "config": {"workload": "%s B%d L%d s_q%d" % (wl.name, B, wl.seq_len, d.s_q), "batch": B,
                    "seq_len": wl.seq_len, "s_q": d.s_q, "n_h": d.n_h, "G": d.G, "d_nope": d.d_nope,
                    "d_rope": d.d_rope, "d_v": d.d_v, "r": d.r,
-                   "step": "expand s_q new tokens + absorb decode + GQA decode",
+                   "step": ("append s_q new tokens to the latent cache + expand them + absorb decode + "
+                            "GQA decode"),
                    "launch": ("cuda_graph replay of the step; absorb path on a second stream, overlapped with "
                               "the tail expansion + GQA path") if graph is not None else "eager, sequential",
                    "eager_ms_per_step": eager_ms,
@@ -425,6 +437,7 @@ def run_ours(args):
         "paths": {"absorb": path_entry(ms_absorb, alg["absorb_bytes"], alg["absorb_flops"]),
                   "gqa": path_entry(ms_gqa, alg["gqa_bytes"], alg["gqa_flops"]),
                   "expand_tail": {"ms": ms_tail},
+                  "append_latent": {"ms": ms_append},
                   "expand_full_cache": {"ms": ms_expand_full, "tflops": exp_flops / (ms_expand_full * 1e-3) / 1e12,
                                         "hbm_gbs": exp_bytes / (ms_expand_full * 1e-3) / 1e9,
                                         "tc_frac": exp_flops / (ms_expand_full * 1e-3) / (tf_burst * 1e12)}},

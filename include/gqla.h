@@ -128,6 +128,23 @@ gqla_status gqla_expand_cache(const gqla_dims* dims, const gqla_kv_layout* layou
                               void* k_pool, void* v_pool, int32_t tail_tokens,
                               int32_t* dev_status, void* stream);
 
+/* Decode-time cache append: the per-step write of the new tokens before the
+ * attention ("GQLA" chatpaper.ai Abstract: the absorb path caches the joint
+ * latent, the GQA path a per-group expanded cache).  For every sequence b the
+ * s_q rows new_rows[b, i, :] = [c_KV (r) ; k_rope (d_rope)] are written to
+ * token positions seq_lens[b] - s_q + i of the latent pool (seq_lens already
+ * count the new tokens), and, when k_pool and v_pool are given, those tokens
+ * are expanded into the per-group pools as gqla_expand_cache does.
+ *   new_rows  device [B, s_q, r + d_rope]
+ *   latent    device pool (written at the new positions only)
+ *   W_uk, W_uv, k_pool, v_pool  as for gqla_expand_cache; k_pool/v_pool may
+ *             both be NULL (absorb-only cache), then W_uk/W_uv are unused.
+ * A sequence shorter than s_q, longer than its slots or with a page outside
+ * the pool is skipped and flagged in *dev_status. */
+gqla_status gqla_append_tokens(const gqla_dims* dims, const gqla_kv_layout* layout, const void* new_rows,
+                               void* latent, const void* W_uk, const void* W_uv, void* k_pool,
+                               void* v_pool, int32_t* dev_status, void* stream);
+
 /* MQA-absorb decode ("GQLA" chatpaper.ai Abstract: an MQA-absorb path
  * identical to MLA's).  Per head: q~ = W_uk^g q_nope, scores
  * scale*(<q~, c_t> + <q_rope, k_rope_t>), latent output sum_t p_t c_t, then

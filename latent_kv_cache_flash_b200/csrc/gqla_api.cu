@@ -262,6 +262,27 @@ gqla_status gqla_expand_cache(const gqla_dims* dims, const gqla_kv_layout* layou
   return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;
 }
 
+gqla_status gqla_append_tokens(const gqla_dims* dims, const gqla_kv_layout* layout, const void* new_rows,
+                               void* latent, const void* W_uk, const void* W_uv, void* k_pool, void* v_pool,
+                               int32_t* dev_status, void* stream) {
+  Problem p;
+  gqla_status s = make_problem(dims, layout, 1, GQLA_PATH_GQA, &p);
+  if (s != GQLA_OK) return s;
+  if (!new_rows || !latent) return GQLA_ERR_INVALID_ARG;
+  const bool expand = k_pool || v_pool;
+  if (expand && (!k_pool || !v_pool || !W_uk || !W_uv)) return GQLA_ERR_INVALID_ARG;
+  if (!aligned16(new_rows) || !aligned16(latent)) return GQLA_ERR_ALIGNMENT;
+  if (expand && (!aligned16(W_uk) || !aligned16(W_uv) || !aligned16(k_pool) || !aligned16(v_pool)))
+    return GQLA_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = append_rows(p, new_rows, latent, dev_status, st);
+  if (e == cudaSuccess && expand) {
+    if (tc_expand_supports(p)) e = tc_expand(p, latent, W_uk, W_uv, k_pool, v_pool, p.d.s_q, dev_status, st);
+    else e = simt_expand(p, latent, W_uk, W_uv, k_pool, v_pool, p.d.s_q, dev_status, st);
+  }
+  return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;
+}
+
 gqla_status gqla_splitkv_combine(int32_t num_splits, int32_t rows, int32_t D, const float* o_part,
                                  const float* lse_part, void* out, gqla_dtype out_dtype, float* lse_out,
                                  void* stream) {

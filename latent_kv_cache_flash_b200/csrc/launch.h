@@ -52,6 +52,8 @@ cudaError_t simt_decode(const Problem& p, gqla_path path, const void* q, const f
                         float* lse, int32_t* st, cudaStream_t s);
 cudaError_t simt_up_proj(const Problem& p, const float* o_lat, const void* W_uv, void* out,
                          cudaStream_t s);
+// Scatter of the step's new latent rows into the pool (append.cu).
+cudaError_t append_rows(const Problem& p, const void* new_rows, void* latent, int32_t* st, cudaStream_t s);
 cudaError_t combine(int S, long long rows, int D, const float* o_part, const float* lse_part,
                     void* out, gqla_dtype out_dtype, float* lse_out, cudaStream_t s);
 

@@ -57,6 +57,7 @@ def lib():
         L.gqla_decode_gqa.argtypes = [pd, pl, P, P, P, P, P, I32, P, SZ, P, P]
         L.gqla_decode_gqa_noalloc.argtypes = [pd, pl, P, P, P, P, P, I32, P, P]
         L.gqla_splitkv_combine.argtypes = [I32, I32, I32, P, P, P, ctypes.c_int, P, P]
+        L.gqla_append_tokens.argtypes = [pd, pl, P, P, P, P, P, P, P, P]
         L.gqla_workspace_bytes.argtypes = [pd, pl, I32, ctypes.c_int]
         L.gqla_workspace_bytes.restype = SZ
         L.gqla_num_splits.argtypes = [pd, pl, I32, ctypes.c_int]
@@ -68,7 +69,7 @@ def lib():
         L.gqla_version.restype = ctypes.c_char_p
         L.gqla_launch_counter.restype = ctypes.c_uint64
         for name in ("gqla_expand_cache", "gqla_decode_absorb", "gqla_decode_gqa", "gqla_decode_gqa_noalloc",
-                     "gqla_splitkv_combine"):
+                     "gqla_splitkv_combine", "gqla_append_tokens"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -144,6 +145,14 @@ def gqla_expand_cache(dims, layout, latent, W_uk, W_uv, k_pool, v_pool, tail_tok
                                 _ptr(k_pool), _ptr(v_pool), int(tail_tokens), _ptr(dev_status),
                                 _stream(stream, latent.device))
     _check(s, "gqla_expand_cache")
+
+
+def gqla_append_tokens(dims, layout, new_rows, latent, W_uk=None, W_uv=None, k_pool=None, v_pool=None,
+                       dev_status=None, stream=None):
+    s = lib().gqla_append_tokens(ctypes.byref(dims), ctypes.byref(layout), _ptr(new_rows), _ptr(latent), _ptr(W_uk),
+                                 _ptr(W_uv), _ptr(k_pool), _ptr(v_pool), _ptr(dev_status),
+                                 _stream(stream, new_rows.device))
+    _check(s, "gqla_append_tokens")
 
 
 def gqla_decode_absorb(dims, layout, q, latent, W_uk, W_uv, out, lse=None, num_splits=0, workspace=None,

@@ -90,6 +90,13 @@ def test_validation_before_launch(G):
     assert L.gqla_decode_gqa(ctypes.byref(d), ctypes.byref(bad), a, a, a, a, None, 0, a, 1 << 30, None,
                              None) == G.GQLA_ERR_INVALID_ARG
     assert L.gqla_splitkv_combine(0, 4, 8, a, a, a, 0, None, None) == G.GQLA_ERR_INVALID_ARG
+    # append: rows and latent pool are required; the two expanded pools come together
+    assert L.gqla_append_tokens(ctypes.byref(d), ctypes.byref(lay), null, a, a, a, a, a, None,
+                                None) == G.GQLA_ERR_INVALID_ARG
+    assert L.gqla_append_tokens(ctypes.byref(d), ctypes.byref(lay), a, a, a, a, a, null, None,
+                                None) == G.GQLA_ERR_INVALID_ARG
+    assert L.gqla_append_tokens(ctypes.byref(d), ctypes.byref(lay), p, a, null, null, null, null, None,
+                                None) == G.GQLA_ERR_ALIGNMENT
 
 
 def test_split_plan_and_workspace(G):
