@@ -18,6 +18,7 @@ on the same workload, one bounded sample of (sequence, group) units per step.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -72,7 +73,9 @@ def algorithmic(wl):
     absorb_flops = d.n_h * keys * 2 * (2 * d.r + d.d_rope) + wl.batch * d.s_q * d.n_h * 2 * d.r * (d.d_nope + d.d_v)
     gqa_bytes = 2 * T * d.G * (d.d_qk + d.d_v)
     gqa_flops = d.n_h * keys * 2 * (d.d_qk + d.d_v)
-    return dict(absorb_bytes=absorb_bytes, absorb_flops=absorb_flops, gqa_bytes=gqa_bytes, gqa_flops=gqa_flops)
+    gqa_shared_bytes = 2 * T * (d.G * (d.d_nope + d.d_v) + d.d_rope)
+    return dict(absorb_bytes=absorb_bytes, absorb_flops=absorb_flops, gqa_bytes=gqa_bytes, gqa_flops=gqa_flops,
+                gqa_shared_bytes=gqa_shared_bytes)
 
 
 # ---------------------------------------------------------------- clocks ---
@@ -356,6 +359,14 @@ def run_ours(args):
     ms_append = timed(append_latent, reps) / reps
     ms_expand_full = timed(lambda: gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0,
                                                           status), 3) / 3
+    # the GQA call over the same cache with the RoPE key stored once per token
+    # row (a second, smaller K pool; V is shared)
+    dims_s = gqla.make_dims(dataclasses.replace(d, k_shared_rope=True))
+    kp_s = torch.empty(tuple(ks[:2]) + (d.G * d.d_nope + d.d_rope,), dtype=d.torch_dtype, device=dev)
+    gqla.gqla_expand_cache(dims_s, lay, inp.latent, inp.W_uk, inp.W_uv, kp_s, vp, 0, status)
+    ms_gqa_s = timed(lambda: gqla.gqla_decode_gqa(dims_s, lay, inp.q, kp_s, vp, out_g, lse_g, 0, ws_g, status),
+                     reps) / reps
+    del kp_s
 
     # end to end through the public API with host buffers: the step's new
     # inputs (queries and the new tokens' latent rows) go host->device, both
@@ -436,6 +447,7 @@ def run_ours(args):
         "clocks": clk,
         "paths": {"absorb": path_entry(ms_absorb, alg["absorb_bytes"], alg["absorb_flops"]),
                   "gqa": path_entry(ms_gqa, alg["gqa_bytes"], alg["gqa_flops"]),
+                  "gqa_shared_rope": path_entry(ms_gqa_s, alg["gqa_shared_bytes"], alg["gqa_flops"]),
                   "expand_tail": {"ms": ms_tail},
                   "append_latent": {"ms": ms_append},
                   "expand_full_cache": {"ms": ms_expand_full, "tflops": exp_flops / (ms_expand_full * 1e-3) / 1e12,
@@ -486,12 +498,33 @@ def time_paths(inp, reps, hbm, tf_burst, expand=True):
     lens = inp.seq_lens_host
     T = sum(lens)
     keys = sum(sum(L - d.s_q + i + 1 for i in range(d.s_q)) for L in lens)
+    gqa_flops = d.n_h * keys * 2 * (d.d_qk + d.d_v)
     work = {"absorb": (2 * T * (d.r + d.d_rope), d.n_h * keys * 2 * (2 * d.r + d.d_rope)),
-            "gqa": (2 * T * d.G * (d.d_qk + d.d_v), d.n_h * keys * 2 * (d.d_qk + d.d_v))}
+            "gqa": (2 * T * d.G * (d.d_qk + d.d_v), gqa_flops),
+            "gqa_shared_rope": (2 * T * (d.G * (d.d_nope + d.d_v) + d.d_rope), gqa_flops)}
+    dims_s = gqla.make_dims(dataclasses.replace(d, k_shared_rope=True))
+    pools = {"kp": kp}
+
+    def shared_pool():
+        # the shared-RoPE K pool replaces the per-group one (one K pool resident at a time)
+        pools.pop("kp", None)
+        ks_s = tuple(ks[:2]) + (d.G * d.d_nope + d.d_rope,)
+        if expand:
+            kp_s = torch.empty(ks_s, dtype=d.torch_dtype, device=dev)
+            gqla.gqla_expand_cache(dims_s, lay, inp.latent, inp.W_uk, inp.W_uv, kp_s, vp)
+        else:
+            kp_s = synth._randn_chunked(ks_s, g, dev, d.torch_dtype)
+        pools["kp_s"] = kp_s
+
     calls = {"absorb": lambda: gqla.gqla_decode_absorb(dims, lay, inp.q, inp.latent, inp.W_uk, inp.W_uv, out, lse,
                                                         0, ws_a),
-             "gqa": lambda: gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out, lse, 0, ws_g)}
+             "gqa": lambda: gqla.gqla_decode_gqa(dims, lay, inp.q, pools["kp"], vp, out, lse, 0, ws_g),
+             "gqa_shared_rope": lambda: gqla.gqla_decode_gqa(dims_s, lay, inp.q, pools["kp_s"], vp, out, lse, 0,
+                                                             ws_g)}
+    del kp
     for name, fn in calls.items():
+        if name == "gqa_shared_rope":
+            shared_pool()
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
@@ -508,7 +541,8 @@ def time_paths(inp, reps, hbm, tf_burst, expand=True):
                      "roofline_frac": max(t_hbm, t_tc) / (ms * 1e-3), "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
                      "tflops": flops / (ms * 1e-3) / 1e12,
                      "splits": gqla.gqla_num_splits(dims, lay, 0, 0 if name == "absorb" else 1)}
-    del kp, vp
+    pools.clear()
+    del vp
     return res
 
 
@@ -531,7 +565,9 @@ def run_sweep(args):
         line = {"sweep": args.sweep, "workload": wl.name, "G": d.G, "s_q": d.s_q, "batch": wl.batch,
                 "seq_len": wl.seq_len if wl.ragged is None else "ragged %d..%d" % wl.ragged,
                 "page_size": wl.page_size, "absorb": res["absorb"], "gqa": res["gqa"],
+                "gqa_shared_rope": res["gqa_shared_rope"],
                 "faster": "absorb" if res["absorb"]["ms"] < res["gqa"]["ms"] else "gqa",
+                "fastest": min(res, key=lambda k: res[k]["ms"]),
                 "pools": "expanded pools filled with seeded random bf16 (decode timing only)"}
         print(json.dumps(line), flush=True)
         del inp

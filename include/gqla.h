@@ -66,6 +66,18 @@ typedef enum gqla_dtype { GQLA_F32 = 0, GQLA_BF16 = 1 } gqla_dtype;
 
 typedef enum gqla_path { GQLA_PATH_ABSORB = 0, GQLA_PATH_GQA = 1 } gqla_path;
 
+/* Row layout of the expanded K pool of the GQA path.  The decoupled RoPE key
+ * is one vector per token shared by every head ("GQLA" scholarbro.com
+ * Abstract: a shared decoupled-RoPE key beside the joint latent), so a K row
+ * may either repeat it in every group or hold it once:
+ *   GQLA_K_PER_GROUP    row = G x [k_nope (d_nope) ; k_rope (d_rope)]
+ *                       (every group is a plain GQA key head of d_nope+d_rope)
+ *   GQLA_K_SHARED_ROPE  row = [G x k_nope (d_nope) ; k_rope (d_rope)]
+ *                       (G*d_nope + d_rope elements: at G = 16, 2112 instead
+ *                       of 3072 per token, 4160 instead of 5120 with V)
+ * Both give the same scores; the second streams fewer bytes. */
+typedef enum gqla_k_layout { GQLA_K_PER_GROUP = 0, GQLA_K_SHARED_ROPE = 1 } gqla_k_layout;
+
 /* Device status bits written to *dev_status (OR-ed). */
 #define GQLA_DEV_SHORT_SEQ 1   /* seq_lens[b] < s_q (or < 0): rows of b zeroed  */
 #define GQLA_DEV_OVERFLOW 2    /* seq_lens[b] above the sequence's token slots  */
@@ -87,6 +99,8 @@ typedef struct gqla_dims {
   int32_t s_q;      /* new tokens per sequence, 1..4                 */
   float scale;      /* softmax scale                                 */
   gqla_dtype dtype; /* element type of q, caches, weights and out    */
+  int32_t k_layout; /* gqla_k_layout of the expanded K pool (GQA path
+                       and expansion; 0 = GQLA_K_PER_GROUP)            */
 } gqla_dims;
 
 /* Where token t of sequence b lives in a token pool (the same geometry serves
@@ -114,12 +128,14 @@ typedef struct gqla_kv_layout {
 /* Per-group cache expansion, the GQA path's precondition ("GQLA" chatpaper.ai
  * Abstract: a GQA path with a per-group expanded cache):
  *   K[b,t,g,:] = [ c_{b,t} W_uk^g ; k_rope_{b,t} ],  V[b,t,g,:] = c_{b,t} W_uv^g
+ * (with GQLA_K_SHARED_ROPE the k_rope part is stored once per token row)
  * for tokens t in [max(0, seq_lens[b] - tail_tokens), seq_lens[b]) of every
  * sequence (tail_tokens <= 0: all tokens).  tail_tokens = s_q expands just the
  * tokens appended by one decode step.
  *   latent  device, pool with rows of r + d_rope elements
  *   W_uk    device [G, r, d_nope];  W_uv device [G, r, d_v]
- *   k_pool  device, pool with rows of G*(d_nope+d_rope) elements (written)
+ *   k_pool  device, pool with rows of G*(d_nope+d_rope) elements, or
+ *           G*d_nope + d_rope with GQLA_K_SHARED_ROPE (written)
  *   v_pool  device, pool with rows of G*d_v elements (written)
  * All three pools use `layout`.  Rows outside the expanded range are not
  * touched. */
@@ -168,7 +184,8 @@ gqla_status gqla_decode_absorb(const gqla_dims* dims, const gqla_kv_layout* layo
  * section "Fonctionnement de la GQA": every head of group g attends over the
  * group's K/V).
  *   q       device [B, s_q, n_h, d_nope + d_rope]
- *   k_pool  device pool, rows of G*(d_nope+d_rope);  v_pool rows of G*d_v
+ *   k_pool  device pool, rows of G*(d_nope+d_rope) (G*d_nope + d_rope with
+ *           GQLA_K_SHARED_ROPE);  v_pool rows of G*d_v
  *   out, lse, num_splits, workspace as for gqla_decode_absorb (path GQA). */
 gqla_status gqla_decode_gqa(const gqla_dims* dims, const gqla_kv_layout* layout,
                             const void* q, const void* k_pool, const void* v_pool,
@@ -220,7 +237,8 @@ int32_t gqla_num_splits(const gqla_dims* dims, const gqla_kv_layout* layout,
                         int32_t num_splits, gqla_path path);
 
 /* Cached bytes per token per layer: absorb path (r + d_rope) elements, GQA
- * path G*(d_nope + d_rope + d_v) elements, times the element size.  At
+ * path G*(d_nope + d_rope + d_v) elements (G*(d_nope + d_v) + d_rope with
+ * GQLA_K_SHARED_ROPE), times the element size.  At
  * LLaMA-3-8B shapes the absorb cache is (512+64)/(2*8*128) = 28.125 % of a
  * GQA baseline with 8 KV heads of 128 ("GQLA" chatpaper.ai Abstract). */
 size_t gqla_cache_bytes_per_token(const gqla_dims* dims, gqla_path path);

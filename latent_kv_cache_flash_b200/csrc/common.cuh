@@ -51,6 +51,15 @@ __device__ __forceinline__ int seq_len_checked(const KvLayout& ly, int b, int s_
   return L;
 }
 
+// Row layout of the expanded K pool (gqla_k_layout): elements per token row,
+// and where group g's parts start in it: d_nope part at g * gs, RoPE part at
+// rope + g * rope_gs (rope_gs = 0 when the RoPE key is stored once).
+struct KRow {
+  int pitch, gs, rope, rope_gs;
+  __host__ __device__ int nope_at(int g) const { return g * gs; }
+  __host__ __device__ int rope_at(int g) const { return rope + g * rope_gs; }
+};
+
 // Pool row of token (b, t); -1 (flagged) for a page id outside the pool.
 __device__ __forceinline__ long long token_row(const KvLayout& ly, int b, int t, int32_t* st) {
   if (ly.page_size == 0) return (long long)b * ly.capacity + t;

@@ -26,6 +26,7 @@ gqla_status check_dims(const gqla_dims* d) {
   if (d->s_q < 1 || d->s_q > 4) return GQLA_ERR_INVALID_ARG;
   if (!(d->scale == d->scale) || isinf(d->scale)) return GQLA_ERR_INVALID_ARG;
   if (d->dtype != GQLA_F32 && d->dtype != GQLA_BF16) return GQLA_ERR_INVALID_ARG;
+  if (d->k_layout != GQLA_K_PER_GROUP && d->k_layout != GQLA_K_SHARED_ROPE) return GQLA_ERR_INVALID_ARG;
   return GQLA_OK;
 }
 
@@ -125,6 +126,10 @@ gqla_status make_problem(const gqla_dims* dims, const gqla_kv_layout* layout, in
   p->d_qk = dims->d_nope + dims->d_rope;
   p->E = dims->r + dims->d_rope;
   p->rows = (long long)layout->batch * dims->s_q * dims->n_h;
+  if (dims->k_layout == GQLA_K_SHARED_ROPE)
+    p->kr = KRow{dims->G * dims->d_nope + dims->d_rope, dims->d_nope, dims->G * dims->d_nope, 0};
+  else
+    p->kr = KRow{dims->G * p->d_qk, p->d_qk, dims->d_nope, p->d_qk};
   p->plan = SplitPlan{1, layout->max_seq_len};
   const bool tc = path == GQLA_PATH_ABSORB ? tc_absorb_supports(*p) : tc_gqa_supports(*p);
   p->plan = make_plan(*dims, *layout, num_splits, path, tc);
@@ -228,7 +233,11 @@ size_t gqla_cache_bytes_per_token(const gqla_dims* dims, gqla_path path) {
   if (check_dims(dims) != GQLA_OK) return 0;
   size_t e = esize(dims->dtype);
   if (path == GQLA_PATH_ABSORB) return (size_t)(dims->r + dims->d_rope) * e;
-  if (path == GQLA_PATH_GQA) return (size_t)dims->G * (dims->d_nope + dims->d_rope + dims->d_v) * e;
+  if (path == GQLA_PATH_GQA) {
+    const size_t k = dims->k_layout == GQLA_K_SHARED_ROPE ? (size_t)dims->G * dims->d_nope + dims->d_rope
+                                                          : (size_t)dims->G * (dims->d_nope + dims->d_rope);
+    return (k + (size_t)dims->G * dims->d_v) * e;
+  }
   return 0;
 }
 

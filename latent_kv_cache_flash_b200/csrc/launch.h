@@ -19,6 +19,7 @@ struct Problem {
   int d_qk;     // d_nope + d_rope
   int E;        // latent row width r + d_rope
   long long rows;  // B * s_q * n_h output rows
+  KRow kr;         // expanded K pool row layout
   SplitPlan plan;
 };
 

@@ -22,7 +22,7 @@ constexpr int kExpandTokens = 16;
 // Block = (16-token block, sequence, group); threads stride the output columns.
 template <typename T>
 __global__ void expand_kernel(KvLayout ly, const T* __restrict__ latent, const T* __restrict__ W_uk,
-                              const T* __restrict__ W_uv, T* __restrict__ kp, T* __restrict__ vp,
+                              const T* __restrict__ W_uv, T* __restrict__ kp, T* __restrict__ vp, KRow kr,
                               int G, int d_n, int d_r, int d_v, int r, int tail, int32_t* st) {
   extern __shared__ float sc[];  // [kExpandTokens][r]
   __shared__ long long srow[kExpandTokens];
@@ -46,7 +46,6 @@ __global__ void expand_kernel(KvLayout ly, const T* __restrict__ latent, const T
     sc[tt * r + k] = row < 0 ? 0.f : to_f32(latent[row * E + k]);
   }
   __syncthreads();
-  const int D_qk = d_n + d_r;
   for (int j = threadIdx.x; j < d_n + d_v; j += blockDim.x) {
     const bool isk = j < d_n;
     const T* W = isk ? (W_uk + (size_t)g * r * d_n + j) : (W_uv + (size_t)g * r * d_v + (j - d_n));
@@ -62,14 +61,17 @@ __global__ void expand_kernel(KvLayout ly, const T* __restrict__ latent, const T
     for (int tt = 0; tt < nt; ++tt) {
       long long row = srow[tt];
       if (row < 0) continue;
-      if (isk) kp[(row * G + g) * D_qk + j] = from_f32<T>(acc[tt]);
+      if (isk) kp[row * kr.pitch + kr.nope_at(g) + j] = from_f32<T>(acc[tt]);
       else vp[(row * G + g) * d_v + (j - d_n)] = from_f32<T>(acc[tt]);
     }
   }
-  for (int i = threadIdx.x; i < nt * d_r; i += blockDim.x) {
-    int tt = i / d_r, a = i % d_r;
-    long long row = srow[tt];
-    if (row >= 0) kp[(row * G + g) * D_qk + d_n + a] = latent[row * E + r + a];
+  // the RoPE key: in every group's part, or once per row (written by group 0)
+  if (kr.rope_gs != 0 || g == 0) {
+    for (int i = threadIdx.x; i < nt * d_r; i += blockDim.x) {
+      int tt = i / d_r, a = i % d_r;
+      long long row = srow[tt];
+      if (row >= 0) kp[row * kr.pitch + kr.rope_at(g) + a] = latent[row * E + r + a];
+    }
   }
 }
 
@@ -95,7 +97,7 @@ __global__ void absorb_q_kernel(const T* __restrict__ q, const T* __restrict__ W
 // split's tokens.  Block = (split, sequence * G + group).
 template <typename T, bool ABSORB>
 __global__ void decode_kernel(KvLayout ly, SplitPlan plan, const T* __restrict__ q, const float* __restrict__ qt,
-                              const T* __restrict__ kpool, const T* __restrict__ vpool,
+                              const T* __restrict__ kpool, const T* __restrict__ vpool, KRow kr,
                               int n_h, int G, int s_q, int d_n, int d_r, int d_v, int r, float scale,
                               T* __restrict__ out_T, float* __restrict__ o_f32, float* __restrict__ lse_dst,
                               long long rows, int32_t* st) {
@@ -106,9 +108,12 @@ __global__ void decode_kernel(KvLayout ly, SplitPlan plan, const T* __restrict__
   const int d_qk = d_n + d_r;
   const int Dk = ABSORB ? (r + d_r) : d_qk;           // key width
   const int Dv = ABSORB ? r : d_v;                    // value width
-  const long long krs = ABSORB ? (long long)(r + d_r) : (long long)G * d_qk;  // key row stride
+  // key element j of a token row: j < ksplit at koff + j, else at kro + (j - ksplit)
+  const long long krs = ABSORB ? (long long)(r + d_r) : (long long)kr.pitch;  // key row stride
   const long long vrs = ABSORB ? (long long)(r + d_r) : (long long)G * d_v;
-  const int koff = ABSORB ? 0 : g * d_qk;
+  const int ksplit = ABSORB ? r : d_n;
+  const int koff = ABSORB ? 0 : kr.nope_at(g);
+  const int kro = ABSORB ? r : kr.rope_at(g);
   const int voff = ABSORB ? 0 : g * d_v;
   int L = seq_len_checked(ly, b, s_q, (split == 0 && g == 0) ? st : nullptr);
   if (!seq_pages_ok(ly, b, L, st)) L = -1;
@@ -138,12 +143,12 @@ __global__ void decode_kernel(KvLayout ly, SplitPlan plan, const T* __restrict__
     for (int t = t_begin; !bad && t < t_end; ++t) {
       long long tr = token_row(ly, b, t, st);
       if (tr < 0) { bad = true; break; }
-      const T* kr = kpool + tr * krs + koff;
+      const T* krow = kpool + tr * krs;
       float part = 0.f;
 #pragma unroll
       for (int u = 0; u < kMaxKeyPerLane; ++u) {
         int j = lane + 32 * u;
-        if (j < Dk) part = fmaf(qv[u], to_f32(kr[j]), part);
+        if (j < Dk) part = fmaf(qv[u], to_f32(krow[j < ksplit ? koff + j : kro + (j - ksplit)]), part);
       }
       const float s = warp_sum(part) * scale;
       const float mn = fmaxf(mx, s);
@@ -229,12 +234,13 @@ cudaError_t simt_expand(const Problem& p, const void* latent, const void* W_uk, 
     auto k = expand_kernel<float>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k<<<grid, 256, smem, s>>>(p.ly, (const float*)latent, (const float*)W_uk, (const float*)W_uv,
-                              (float*)k_pool, (float*)v_pool, d.G, d.d_nope, d.d_rope, d.d_v, d.r, tail, st);
+                              (float*)k_pool, (float*)v_pool, p.kr, d.G, d.d_nope, d.d_rope, d.d_v, d.r, tail,
+                              st);
   } else {
     auto k = expand_kernel<__nv_bfloat16>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k<<<grid, 256, smem, s>>>(p.ly, (const __nv_bfloat16*)latent, (const __nv_bfloat16*)W_uk,
-                              (const __nv_bfloat16*)W_uv, (__nv_bfloat16*)k_pool, (__nv_bfloat16*)v_pool,
+                              (const __nv_bfloat16*)W_uv, (__nv_bfloat16*)k_pool, (__nv_bfloat16*)v_pool, p.kr,
                               d.G, d.d_nope, d.d_rope, d.d_v, d.r, tail, st);
   }
   count_launch();
@@ -270,8 +276,9 @@ cudaError_t simt_decode(const Problem& p, gqla_path path, const void* q, const f
   const int threads = 128;
 #define GQLA_DEC(T, AB)                                                                                   \
   decode_kernel<T, AB><<<grid, threads, 0, s>>>(p.ly, p.plan, (const T*)q, qt, (const T*)kpool,           \
-                                                (const T*)vpool, d.n_h, d.G, d.s_q, d.d_nope, d.d_rope,   \
-                                                d.d_v, d.r, d.scale, (T*)out_T, o_f32, lse, p.rows, st)
+                                                (const T*)vpool, p.kr, d.n_h, d.G, d.s_q, d.d_nope,       \
+                                                d.d_rope, d.d_v, d.r, d.scale, (T*)out_T, o_f32, lse,     \
+                                                p.rows, st)
   if (d.dtype == GQLA_F32) {
     if (path == GQLA_PATH_ABSORB) GQLA_DEC(float, true); else GQLA_DEC(float, false);
   } else {

@@ -3,7 +3,17 @@
 
 #include "launch.h"
 
+#include <cuda.h>
+
 namespace gqla {
+
+// Row-major [rows, cols] bf16 tensor map, 64-column x box_rows boxes, 128-byte
+// swizzle (tmap.cu).  cols * 2 and row_pitch_elems * 2 must be multiples of 16.
+bool tmap_bf16_sw128(CUtensorMap* map, const void* base, long long cols, long long rows, long long row_pitch_elems,
+                     int box_rows);
+// The expanded K and V pools as [pool row, row width] maps with 64 x 64 boxes;
+// a group's d_nope / RoPE / V chunks sit at column offsets given by p.kr.
+bool gqa_pool_maps(const Problem& p, const void* k_pool, const void* v_pool, CUtensorMap* kmap, CUtensorMap* vmap);
 
 // GQA decode over the expanded cache: mma.sync bf16 tiles, cp.async.bulk
 // staged K/V pages, online softmax per 16-row block.

@@ -387,36 +387,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)f;
-  }
-  return fn;
-}
-
-// Row-major [rows, cols] bf16 matrix, boxes of 64 columns x box_rows rows, 128-byte swizzle.
-bool make_2d_map(CUtensorMap* map, const void* base, long long cols, long long rows, long long row_pitch_elems,
-                 int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t gstride[1] = {(cuuint64_t)row_pitch_elems * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool tc_absorb_supports(const Problem& p) {
@@ -441,7 +411,7 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
   long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
                                         : (long long)p.ly.num_pages * p.ly.page_size;
   CUtensorMap kv_map;
-  if (!make_2d_map(&kv_map, latent, kE, nrows, kE, kTk)) return cudaErrorInvalidValue;
+  if (!tmap_bf16_sw128(&kv_map, latent, kE, nrows, kE, kTk)) return cudaErrorInvalidValue;
   AbsorbParams prm;
   prm.ly = p.ly;
   prm.plan = p.plan;

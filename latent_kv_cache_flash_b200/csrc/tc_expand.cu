@@ -41,6 +41,7 @@ constexpr int kThreads = 6 * 32;
 struct ExpandParams {
   KvLayout ly;
   bf16* kp;
+  KRow kr;
   bf16* vp;
   const bf16* latent;
   int G;
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_ld32(tl + (uint32_t)(ab * kN + 32 * c), v);
           ptx::tmem_ld_wait();
           if (write) {
-            bf16* dst = c < kDn / 32 ? p.kp + (row * G + g) * (kDn + kDr) + 32 * c
+            bf16* dst = c < kDn / 32 ? p.kp + row * p.kr.pitch + p.kr.nope_at(g) + 32 * c
                                      : p.vp + (row * G + g) * kDv + 32 * (c - kDn / 32);
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
@@ -236,9 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (write) {
+        if (write && (p.kr.rope_gs != 0 || g == 0)) {   // a shared RoPE key is written by group 0
           const uint4* src = reinterpret_cast<const uint4*>(p.latent + row * kE + kR);
-          uint4* dst = reinterpret_cast<uint4*>(p.kp + (row * G + g) * (kDn + kDr) + kDn);
+          uint4* dst = reinterpret_cast<uint4*>(p.kp + row * p.kr.pitch + p.kr.rope_at(g));
 #pragma unroll
           for (int e = 0; e < kDr / 8; ++e) dst[e] = src[e];
         }
@@ -256,34 +257,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)f;
-  }
-  return fn;
-}
-
-bool map_2d(CUtensorMap* map, const void* base, long long cols, long long rows, long long pitch, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t gstride[1] = {(cuuint64_t)pitch * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -304,12 +277,14 @@ cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, co
   const long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
                                               : (long long)p.ly.num_pages * p.ly.page_size;
   CUtensorMap lat_map, uk_map, uv_map;
-  if (!map_2d(&lat_map, latent, kE, nrows, kE, 64) || !map_2d(&uk_map, W_uk, kDn, (long long)d.G * kR, kDn, kKC) ||
-      !map_2d(&uv_map, W_uv, kDv, (long long)d.G * kR, kDv, kKC))
+  if (!tmap_bf16_sw128(&lat_map, latent, kE, nrows, kE, 64) ||
+      !tmap_bf16_sw128(&uk_map, W_uk, kDn, (long long)d.G * kR, kDn, kKC) ||
+      !tmap_bf16_sw128(&uv_map, W_uv, kDv, (long long)d.G * kR, kDv, kKC))
     return cudaErrorInvalidValue;
   ExpandParams prm;
   prm.ly = p.ly;
   prm.kp = (bf16*)k_pool;
+  prm.kr = p.kr;
   prm.vp = (bf16*)v_pool;
   prm.latent = (const bf16*)latent;
   prm.G = d.G;

@@ -8,9 +8,10 @@
 // d_qk = 192, d_v = 128), so the kernel is built around moving those bytes:
 //
 //  * one CTA per (key-range split, sequence, group[, 64-row block]);
-//  * a producer warp streams 64-token K and V tiles with TMA (3-D tensor maps
-//    over the pool's [token row, group, dim] view, 128-byte swizzle) into a
-//    2-stage mbarrier ring; two CTAs fit on an SM;
+//  * a producer warp streams 64-token K and V tiles with TMA (2-D tensor maps
+//    over the pools' token rows, 128-byte swizzle; the group's chunks are
+//    column offsets, so a RoPE key stored once per row is read from there)
+//    into a 2-stage mbarrier ring; two CTAs fit on an SM;
 //  * four consumer warps each take 16 tokens of a tile (or, for more than 16
 //    rows, one 16-row block each), compute S = Q K^T and O += P V with
 //    mma.sync m16n8k16 bf16 (fp32 accumulate) from ldmatrix'd fragments, and
@@ -49,6 +50,7 @@ struct GqaParams {
   int n_h, G, m, s_q;
   int rows_unit;   // m * s_q rows of one (sequence, group)
   int rbc;         // 16-row blocks per CTA: 1, 2 or 4
+  KRow kr;         // K pool row layout
   float scale_log2;
   long long rows;  // B * s_q * n_h
   int32_t* st;
@@ -90,6 +92,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       ptx::prefetch_tmap(&kmap);
       ptx::prefetch_tmap(&vmap);
+      const int kx = p.kr.nope_at(g), kxr = p.kr.rope_at(g), vx = g * kDv;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kStages, k = j / kStages;
         if (k > 0 && !ptx::mbar_wait(&empty_bar[s], (k - 1) & 1)) {
@@ -102,11 +105,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int row0 = (int)token_row(p.ly, b, t0, nullptr);
         uint8_t* st = smem + s * kStageBytes;
         ptx::mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
-#pragma unroll
-        for (int c = 0; c < kKChunks; ++c) ptx::tma_load_3d(st + c * kChunkBytes, &kmap, &full_bar[s], 64 * c, g, row0);
+        // K: the group's two d_nope chunks, then its RoPE chunk; V: two chunks
+        ptx::tma_load_2d(st, &kmap, &full_bar[s], kx, row0);
+        ptx::tma_load_2d(st + kChunkBytes, &kmap, &full_bar[s], kx + 64, row0);
+        ptx::tma_load_2d(st + 2 * kChunkBytes, &kmap, &full_bar[s], kxr, row0);
 #pragma unroll
         for (int c = 0; c < kVChunks; ++c)
-          ptx::tma_load_3d(st + (kKChunks + c) * kChunkBytes, &vmap, &full_bar[s], 64 * c, g, row0);
+          ptx::tma_load_2d(st + (kKChunks + c) * kChunkBytes, &vmap, &full_bar[s], vx + 64 * c, row0);
       }
     }
     return;
@@ -317,36 +322,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)f;
-  }
-  return fn;
-}
-
-// [dim (inner), group, token row] view of a per-group pool, 64x1x64 boxes.
-bool make_pool_map(CUtensorMap* map, const void* base, int dim, int G, long long nrows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gdim[3] = {(cuuint64_t)dim, (cuuint64_t)G, (cuuint64_t)nrows};
-  cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * 2 * G};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kT};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool tc_gqa_supports(const Problem& p) {
@@ -362,11 +337,8 @@ cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, c
                           float* o_part, float* lse_dst, int32_t* st, cudaStream_t s) {
   if (tc_gqa_wide_supports(p)) return tc_gqa_wide_decode(p, q, k_pool, v_pool, out, o_part, lse_dst, st, s);
   const auto& d = p.d;
-  long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
-                                        : (long long)p.ly.num_pages * p.ly.page_size;
   CUtensorMap kmap, vmap;
-  if (!make_pool_map(&kmap, k_pool, kDqk, d.G, nrows) || !make_pool_map(&vmap, v_pool, kDv, d.G, nrows))
-    return cudaErrorInvalidValue;
+  if (!gqa_pool_maps(p, k_pool, v_pool, &kmap, &vmap)) return cudaErrorInvalidValue;
   GqaParams prm;
   prm.ly = p.ly;
   prm.plan = p.plan;
@@ -384,6 +356,7 @@ cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, c
   prm.scale_log2 = d.scale * 1.4426950408889634f;
   prm.rows = p.rows;
   prm.st = st;
+  prm.kr = p.kr;
   dim3 grid(p.plan.num_splits, p.ly.batch * d.G, (rb + prm.rbc - 1) / prm.rbc);
   cudaError_t e = ensure_smem_limit((const void*)gqa_decode_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;

@@ -10,7 +10,8 @@
 // One CTA per (key-range split, sequence, group, block of 128 rows):
 //  * the 128 x 192 query tile is gathered into 128-byte-swizzled shared
 //    memory once; 64-token K (64 x 192) and V (64 x 128) tiles stream in with
-//    TMA (3-D views of the pools) into a 4-stage mbarrier ring;
+//    TMA (2-D maps over the pools' token rows; a group's chunks are column
+//    offsets) into a 4-stage mbarrier ring;
 //  * warp 1 issues S = Q K^T (12 tcgen05.mma, M=128, N=64, K=16) into a
 //    double-buffered S in TMEM; warp 6 issues O += P V (4 tcgen05.mma,
 //    M=128, N=128, K=16, V as an MN-major operand) into O in TMEM;
@@ -54,6 +55,7 @@ struct WideParams {
   int n_h, G, m, s_q;
   int rows_unit;      // m * s_q
   int rblocks;        // ceil(rows_unit / 128)
+  KRow kr;            // K pool row layout
   float scale_log2;
   long long rows;     // B * s_q * n_h
   int32_t* st;
@@ -124,10 +126,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row0 = (int)token_row(p.ly, b, t_begin + j * kT, nullptr);
         uint8_t* dst = sKV + s * kStageBytes;
         ptx::mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
-        for (int c = 0; c < kKChunks; ++c)
-          ptx::tma_load_3d(dst + c * kChunkBytes, &kmap, &kv_full[s], 64 * c, g, row0);
+        ptx::tma_load_2d(dst, &kmap, &kv_full[s], p.kr.nope_at(g), row0);
+        ptx::tma_load_2d(dst + kChunkBytes, &kmap, &kv_full[s], p.kr.nope_at(g) + 64, row0);
+        ptx::tma_load_2d(dst + 2 * kChunkBytes, &kmap, &kv_full[s], p.kr.rope_at(g), row0);
         for (int c = 0; c < kVChunks; ++c)
-          ptx::tma_load_3d(dst + (kKChunks + c) * kChunkBytes, &vmap, &kv_full[s], 64 * c, g, row0);
+          ptx::tma_load_2d(dst + (kKChunks + c) * kChunkBytes, &vmap, &kv_full[s], g * kDv + 64 * c, row0);
         issued = j + 1;
       }
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
@@ -352,34 +355,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)f;
-  }
-  return fn;
-}
-
-bool pool_map(CUtensorMap* map, const void* base, int dim, int G, long long nrows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gdim[3] = {(cuuint64_t)dim, (cuuint64_t)G, (cuuint64_t)nrows};
-  cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * 2 * G};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kT};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool tc_gqa_wide_supports(const Problem& p) {
@@ -394,11 +369,8 @@ bool tc_gqa_wide_supports(const Problem& p) {
 cudaError_t tc_gqa_wide_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
                                float* o_part, float* lse_dst, int32_t* st, cudaStream_t s) {
   const auto& d = p.d;
-  const long long nrows = p.ly.page_size == 0 ? (long long)p.ly.batch * p.ly.capacity
-                                              : (long long)p.ly.num_pages * p.ly.page_size;
   CUtensorMap kmap, vmap;
-  if (!pool_map(&kmap, k_pool, kDqk, d.G, nrows) || !pool_map(&vmap, v_pool, kDv, d.G, nrows))
-    return cudaErrorInvalidValue;
+  if (!gqa_pool_maps(p, k_pool, v_pool, &kmap, &vmap)) return cudaErrorInvalidValue;
   WideParams prm;
   prm.ly = p.ly;
   prm.plan = p.plan;
@@ -415,6 +387,7 @@ cudaError_t tc_gqa_wide_decode(const Problem& p, const void* q, const void* k_po
   prm.scale_log2 = d.scale * 1.4426950408889634f;
   prm.rows = p.rows;
   prm.st = st;
+  prm.kr = p.kr;
   cudaError_t e = ensure_smem_limit((const void*)gqa_wide_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.plan.num_splits, p.ly.batch * d.G, prm.rblocks);

@@ -19,6 +19,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqla.so
 GQLA_OK, GQLA_ERR_INVALID_ARG, GQLA_ERR_UNSUPPORTED, GQLA_ERR_ALIGNMENT, GQLA_ERR_WORKSPACE, GQLA_ERR_CUDA = range(6)
 GQLA_F32, GQLA_BF16 = 0, 1
 GQLA_PATH_ABSORB, GQLA_PATH_GQA = 0, 1
+GQLA_K_PER_GROUP, GQLA_K_SHARED_ROPE = 0, 1
 DEV_SHORT_SEQ, DEV_OVERFLOW, DEV_BAD_PAGE, DEV_TIMEOUT = 1, 2, 4, 8
 
 
@@ -31,7 +32,8 @@ class GqlaError(RuntimeError):
 class GqlaDims(ctypes.Structure):
     _fields_ = [("n_h", ctypes.c_int32), ("G", ctypes.c_int32), ("d_nope", ctypes.c_int32),
                 ("d_rope", ctypes.c_int32), ("d_v", ctypes.c_int32), ("r", ctypes.c_int32),
-                ("s_q", ctypes.c_int32), ("scale", ctypes.c_float), ("dtype", ctypes.c_int)]
+                ("s_q", ctypes.c_int32), ("scale", ctypes.c_float), ("dtype", ctypes.c_int),
+                ("k_layout", ctypes.c_int32)]
 
 
 class GqlaKvLayout(ctypes.Structure):
@@ -94,12 +96,14 @@ def _check(status: int, what: str):
 
 def make_dims(d) -> GqlaDims:
     """Builds the C struct from any object with n_h, G, d_nope, d_rope, d_v, r,
-    s_q, softmax_scale (or scale) and dtype ("f32"/"bf16")."""
+    s_q, softmax_scale (or scale), dtype ("f32"/"bf16") and optionally
+    k_shared_rope (the expanded K pool stores the RoPE key once per token)."""
     scale = getattr(d, "softmax_scale", None)
     if scale is None:
         scale = d.scale
     dt = GQLA_F32 if d.dtype in ("f32", torch.float32) else GQLA_BF16
-    return GqlaDims(d.n_h, d.G, d.d_nope, d.d_rope, d.d_v, d.r, d.s_q, float(scale), dt)
+    kl = GQLA_K_SHARED_ROPE if getattr(d, "k_shared_rope", False) else GQLA_K_PER_GROUP
+    return GqlaDims(d.n_h, d.G, d.d_nope, d.d_rope, d.d_v, d.r, d.s_q, float(scale), dt, kl)
 
 
 def make_layout(seq_lens: torch.Tensor, max_seq_len: int, page_size: int = 0, capacity: int = 0,

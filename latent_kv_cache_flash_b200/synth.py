@@ -36,6 +36,7 @@ class Dims:
     s_q: int = 1
     dtype: str = "bf16"            # "f32" or "bf16"
     scale: Optional[float] = None  # default 1/sqrt(d_nope + d_rope)
+    k_shared_rope: bool = False    # expanded K rows hold the RoPE key once, not per group
 
     @property
     def m(self) -> int:
@@ -194,7 +195,9 @@ def _randn_chunked(shape, gen, dev, tdt, chunk_elems=1 << 28):
 
 def expanded_pool_shapes(inp: Inputs):
     """Shapes of the per-group expanded K and V pools with the latent pool's
-    geometry: token rows [G, d_nope + d_rope] and [G, d_v]."""
+    geometry: token rows [G, d_nope + d_rope] (or [G * d_nope + d_rope] when
+    the RoPE key is stored once) and [G, d_v]."""
     d = inp.dims
     lead = tuple(inp.latent.shape[:2])
-    return lead + (d.G, d.d_qk), lead + (d.G, d.d_v)
+    k = (d.G * d.d_nope + d.d_rope,) if d.k_shared_rope else (d.G, d.d_qk)
+    return lead + k, lead + (d.G, d.d_v)

@@ -40,9 +40,11 @@ def test_status_strings(G):
 
 
 def _dims(mod, **kw):
-    base = dict(n_h=32, G=8, d_nope=128, d_rope=64, d_v=128, r=512, s_q=1, scale=192 ** -0.5, dtype=mod.GQLA_BF16)
+    base = dict(n_h=32, G=8, d_nope=128, d_rope=64, d_v=128, r=512, s_q=1, scale=192 ** -0.5, dtype=mod.GQLA_BF16,
+                k_layout=mod.GQLA_K_PER_GROUP)
     base.update(kw)
-    return mod.GqlaDims(*[base[k] for k in ("n_h", "G", "d_nope", "d_rope", "d_v", "r", "s_q", "scale", "dtype")])
+    return mod.GqlaDims(*[base[k] for k in ("n_h", "G", "d_nope", "d_rope", "d_v", "r", "s_q", "scale", "dtype",
+                                            "k_layout")])
 
 
 def _layout(G, B=4, L=8192, page=0):
@@ -60,6 +62,15 @@ def test_cache_bytes_28_125_percent(G):
     assert absorb / baseline == a["value"]
     # the expanded GQLA cache of the same layer: 8 groups * (192 + 128) bf16
     assert G.gqla_cache_bytes_per_token(d, G.GQLA_PATH_GQA) == 8 * 320 * 2
+    # with the RoPE key stored once per token: 8 * (128 + 128) + 64 elements;
+    # DeepSeek-V3 shapes (G = 16): 4160 instead of 5120 elements per token
+    shared = _dims(G, k_layout=G.GQLA_K_SHARED_ROPE)
+    assert G.gqla_cache_bytes_per_token(shared, G.GQLA_PATH_GQA) == (8 * 256 + 64) * 2
+    assert G.gqla_cache_bytes_per_token(shared, G.GQLA_PATH_ABSORB) == absorb
+    ds = _dims(G, n_h=128, G=16)
+    ds_shared = _dims(G, n_h=128, G=16, k_layout=G.GQLA_K_SHARED_ROPE)
+    assert G.gqla_cache_bytes_per_token(ds, G.GQLA_PATH_GQA) == 5120 * 2
+    assert G.gqla_cache_bytes_per_token(ds_shared, G.GQLA_PATH_GQA) == 4160 * 2
 
 
 def test_validation_before_launch(G):
@@ -70,6 +81,9 @@ def test_validation_before_launch(G):
     s = L.gqla_decode_gqa(ctypes.byref(bad_groups), ctypes.byref(lay), null, null, null, null, None, 0, null, 0,
                           None, None)
     assert s == G.GQLA_ERR_INVALID_ARG
+    d = _dims(G, k_layout=7)     # not a gqla_k_layout
+    assert L.gqla_decode_gqa(ctypes.byref(d), ctypes.byref(lay), null, null, null, null, None, 0, null, 0,
+                             None, None) == G.GQLA_ERR_INVALID_ARG
     d = _dims(G, s_q=5)
     assert L.gqla_decode_absorb(ctypes.byref(d), ctypes.byref(lay), null, null, null, null, null, None, 0, null,
                                 0, None, None) == G.GQLA_ERR_INVALID_ARG
