@@ -558,16 +558,22 @@ def run_sweep(args):
         points = [synth.dsv3(seq_len=L, s_q=s_q) for L in (8192, 16384, 32768, 65536) for s_q in (1, 2)]
     else:
         points = [synth.ragged_paged()]
+    from latent_kv_cache_flash_b200 import gqla
     for wl in points:
         inp = synth.make_inputs(wl, "cuda")
         res = time_paths(inp, max(5, args.steps // 10), hbm, tf_burst, expand=False)
         d = wl.dims
+        lay = gqla.make_layout(inp.seq_lens, inp.max_seq_len, wl.page_size,
+                               inp.capacity if wl.page_size == 0 else 0, inp.block_table, inp.num_pages)
+        sel = gqla.gqla_select_path(gqla.make_dims(d), lay, sum(inp.seq_lens_host))
         line = {"sweep": args.sweep, "workload": wl.name, "G": d.G, "s_q": d.s_q, "batch": wl.batch,
                 "seq_len": wl.seq_len if wl.ragged is None else "ragged %d..%d" % wl.ragged,
                 "page_size": wl.page_size, "absorb": res["absorb"], "gqa": res["gqa"],
                 "gqa_shared_rope": res["gqa_shared_rope"],
                 "faster": "absorb" if res["absorb"]["ms"] < res["gqa"]["ms"] else "gqa",
                 "fastest": min(res, key=lambda k: res[k]["ms"]),
+                "selector": {"path": "gqa" if sel[0] == gqla.GQLA_PATH_GQA else "absorb",
+                             "absorb_ms": sel[1] * 1e-3, "gqa_ms": sel[2] * 1e-3},
                 "pools": "expanded pools filled with seeded random bf16 (decode timing only)"}
         print(json.dumps(line), flush=True)
         del inp

@@ -236,6 +236,34 @@ size_t gqla_workspace_bytes(const gqla_dims* dims, const gqla_kv_layout* layout,
 int32_t gqla_num_splits(const gqla_dims* dims, const gqla_kv_layout* layout,
                         int32_t num_splits, gqla_path path);
 
+/* Hardware figures for gqla_select_path.  NULL selects the library's
+ * defaults: the current device's SM count with the copy bandwidth and dense
+ * bf16 tensor rate measured on a B200. */
+typedef struct gqla_hw {
+  int32_t sms;        /* streaming multiprocessors                      */
+  double hbm_gbs;     /* device-memory copy bandwidth, GB/s              */
+  double tc_tflops;   /* dense bf16 tensor-core rate, TFLOP/s            */
+} gqla_hw;
+
+typedef struct gqla_path_estimate {
+  double absorb_us;   /* predicted device time of gqla_decode_absorb     */
+  double gqa_us;      /* predicted device time of gqla_decode_gqa        */
+  gqla_path path;     /* the faster of the two                           */
+} gqla_path_estimate;
+
+/* Runtime path choice ("GQLA" chatpaper.ai Abstract: the same weights run
+ * either path and the runtime picks the one that suits the hardware).  From
+ * the dims (k_layout included), the layout's batch and max_seq_len, and the
+ * batch's total cached tokens (sum of seq_lens, known to the caller; the
+ * device array is not read), predicts both calls' device times with a model
+ * of this library's kernels (bound resource, tile shape, split plan and
+ * measured efficiency) on the given hardware, and names the faster path.
+ * Host only: launches nothing.  Errors: INVALID_ARG for bad dims or layout,
+ * total_tokens outside [batch * s_q, batch * max_seq_len], or non-positive
+ * hardware figures. */
+gqla_status gqla_select_path(const gqla_dims* dims, const gqla_kv_layout* layout, int64_t total_tokens,
+                             const gqla_hw* hw, gqla_path_estimate* est);
+
 /* Cached bytes per token per layer: absorb path (r + d_rope) elements, GQA
  * path G*(d_nope + d_rope + d_v) elements (G*(d_nope + d_v) + d_rope with
  * GQLA_K_SHARED_ROPE), times the element size.  At

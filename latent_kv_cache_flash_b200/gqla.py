@@ -42,6 +42,14 @@ class GqlaKvLayout(ctypes.Structure):
                 ("max_blocks_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
 
 
+class GqlaHw(ctypes.Structure):
+    _fields_ = [("sms", ctypes.c_int32), ("hbm_gbs", ctypes.c_double), ("tc_tflops", ctypes.c_double)]
+
+
+class GqlaPathEstimate(ctypes.Structure):
+    _fields_ = [("absorb_us", ctypes.c_double), ("gqa_us", ctypes.c_double), ("path", ctypes.c_int)]
+
+
 _lib = None
 
 
@@ -60,6 +68,8 @@ def lib():
         L.gqla_decode_gqa_noalloc.argtypes = [pd, pl, P, P, P, P, P, I32, P, P]
         L.gqla_splitkv_combine.argtypes = [I32, I32, I32, P, P, P, ctypes.c_int, P, P]
         L.gqla_append_tokens.argtypes = [pd, pl, P, P, P, P, P, P, P, P]
+        L.gqla_select_path.argtypes = [pd, pl, ctypes.c_int64, ctypes.POINTER(GqlaHw),
+                                       ctypes.POINTER(GqlaPathEstimate)]
         L.gqla_workspace_bytes.argtypes = [pd, pl, I32, ctypes.c_int]
         L.gqla_workspace_bytes.restype = SZ
         L.gqla_num_splits.argtypes = [pd, pl, I32, ctypes.c_int]
@@ -71,7 +81,7 @@ def lib():
         L.gqla_version.restype = ctypes.c_char_p
         L.gqla_launch_counter.restype = ctypes.c_uint64
         for name in ("gqla_expand_cache", "gqla_decode_absorb", "gqla_decode_gqa", "gqla_decode_gqa_noalloc",
-                     "gqla_splitkv_combine", "gqla_append_tokens"):
+                     "gqla_splitkv_combine", "gqla_append_tokens", "gqla_select_path"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -136,6 +146,15 @@ def gqla_workspace_bytes(dims: GqlaDims, layout: GqlaKvLayout, num_splits: int, 
 
 def gqla_num_splits(dims: GqlaDims, layout: GqlaKvLayout, num_splits: int, path: int) -> int:
     return int(lib().gqla_num_splits(ctypes.byref(dims), ctypes.byref(layout), num_splits, path))
+
+
+def gqla_select_path(dims: GqlaDims, layout: GqlaKvLayout, total_tokens: int, hw: Optional[GqlaHw] = None):
+    """(path, absorb_us, gqa_us): the library's prediction of both decode calls."""
+    est = GqlaPathEstimate()
+    s = lib().gqla_select_path(ctypes.byref(dims), ctypes.byref(layout), int(total_tokens),
+                               ctypes.byref(hw) if hw is not None else None, ctypes.byref(est))
+    _check(s, "gqla_select_path")
+    return int(est.path), float(est.absorb_us), float(est.gqa_us)
 
 
 def workspace_for(dims: GqlaDims, layout: GqlaKvLayout, num_splits: int, path: int, device) -> torch.Tensor:
