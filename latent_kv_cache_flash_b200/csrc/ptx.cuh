@@ -172,6 +172,14 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= (uint64_t)2 << 61;
   return d;
 }
+// The descriptor of a shared-memory address `bytes` (a multiple of 16) past the
+// one `d` describes: the start-address field holds address >> 4 and shared
+// memory ends below 256 KB, so a plain add cannot carry out of the field.  An
+// issue loop that builds each descriptor from scratch spends more cycles per
+// tcgen05.mma than a small MMA takes; with a base descriptor and constant
+// offsets one thread issues at the tensor pipe's rate.
+__device__ __forceinline__ uint64_t umma_desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 // Instruction descriptor of kind::f16: bf16 x bf16 -> f32, dense.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |

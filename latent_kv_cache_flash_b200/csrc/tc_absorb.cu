@@ -21,12 +21,13 @@
 //    tcgen05.mma (M=64, N=256, A = P from shared memory, B = the same latent
 //    tile as an MN-major operand), so a stage is released as soon as its PV
 //    completes;
-//  * warps 2-5 load Q~ into TMEM, then per tile read S rows with tcgen05.ld,
-//    run the online softmax in the log2 domain with lazy rescaling (O is
-//    rescaled only when a row maximum grows by more than 2^8, through the
-//    16-lane TMEM shape so the Q~/S lanes are never touched), write P (bf16)
-//    to shared memory, and at the end stage O through shared memory to write
-//    the fp32 latent output and the log-sum-exp of the split.
+//  * warps 2-5 load Q~ into TMEM, then per tile read S with tcgen05.ld in the
+//    16-lane shape (two threads per row, 32 tokens each, so all 128 threads
+//    work), run the online softmax in the log2 domain with lazy rescaling (O
+//    is rescaled only when a row maximum grows by more than 2^8, through the
+//    same shape so the Q~/S lanes are never touched), write P (bf16) to shared
+//    memory, and at the end stage O through shared memory to write the fp32
+//    latent output and the log-sum-exp of the split.
 #include <math.h>
 
 #include "ptx.cuh"
@@ -159,13 +160,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ptx::tc_fence_after();
         const uint32_t d = tmem + kSCol + (uint32_t)kTk * sb;
-        const uint32_t st_addr = kv_addr + s * kStageBytes;
+        const uint64_t bd0 = ptx::umma_desc_sw128(kv_addr + s * kStageBytes, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kE / 16; ++kk) {
-          const uint32_t koff = (kk >> 2), kin = (kk & 3) * 32;
-          const uint64_t bd = ptx::umma_desc_sw128(st_addr + koff * kKVChunk + kin, 16, 1024);
-          ptx::umma_bf16_ts(d, tmem + 8u * kk, bd, idesc_qk, kk > 0);
-        }
+        for (int kk = 0; kk < kE / 16; ++kk)
+          ptx::umma_bf16_ts(d, tmem + 8u * kk, ptx::umma_desc_add(bd0, (kk >> 2) * kKVChunk + (kk & 3) * 32),
+                            idesc_qk, kk > 0);
         ptx::umma_commit(&s_full[sb]);
       }
       if (!ok) {
@@ -180,22 +179,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- PV issuer
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_pv = ptx::idesc_bf16(kM, 256, false, true);
-      const uint32_t kv_addr = ptx::smem_u32(sKV), p_addr = ptx::smem_u32(sP);
+      const uint32_t kv_addr = ptx::smem_u32(sKV);
+      const uint64_t ad0 = ptx::umma_desc_sw128(ptx::smem_u32(sP), 16, 1024);
       bool ok = true;
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kStages;
         ok = ptx::mbar_wait(&p_full, j & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t st_addr = kv_addr + s * kStageBytes;
+        const uint64_t bd0 = ptx::umma_desc_sw128(kv_addr + s * kStageBytes, kKVChunk, 1024);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
-          for (int kk = 0; kk < kTk / 16; ++kk) {
-            const uint64_t a = ptx::umma_desc_sw128(p_addr + kk * 32, 16, 1024);
-            const uint64_t bd = ptx::umma_desc_sw128(st_addr + (4 * h) * kKVChunk + kk * 16 * 128, kKVChunk, 1024);
-            ptx::umma_bf16(tmem + kOLane + 256u * h, a, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kTk / 16; ++kk)
+            ptx::umma_bf16(tmem + kOLane + 256u * h, ptx::umma_desc_add(ad0, kk * 32),
+                           ptx::umma_desc_add(bd0, (4 * h) * kKVChunk + kk * 16 * 128), idesc_pv,
+                           (j > 0 || kk > 0) ? 1u : 0u);
         }
         ptx::umma_commit(&pv_done);
         ptx::umma_commit(&kv_empty[s]);
@@ -210,21 +209,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------- softmax + epilogue warps
     const int qd = warp & 3;                    // TMEM lane quarter of this warp
-    const int row = 16 * qd + (lane & 15);      // S row held by lanes 0-15
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+    // S and O are read through the 16-lane TMEM shape: thread t holds row
+    // 8 (t % 2) + t / 4 of the quarter and the columns of parity (t / 2) % 2,
+    // so every row is shared by two threads (t and t ^ 2), 32 tokens each.
+    const int o_dp = 8 * (lane & 1) + (lane >> 2);
+    const int half = (lane >> 1) & 1;
+    const int row = 16 * qd + o_dp;
     const int r_local = hb * kM + row;
     const bool in_range = r_local < p.rows_unit;   // rows past the sequence's heads are padding
     const bool valid = in_range && L >= 0;
     const int vis = valid ? L - p.s_q + r_local / (p.rows_unit / p.s_q) + 1 : 0;
-    // lanes 16-31 address O through the 16-lane shape: this thread's O row
-    const int o_dp = 8 * (lane & 1) + (lane >> 2);
 
-    // Q~ = [q~ (512) ; q_rope (64)] of this row into TMEM (lanes 0-15), as
-    // bf16 pairs; lanes 16-31 store zeros into the O half-lanes, which the
-    // first PV overwrites.
+    // Q~ = [q~ (512) ; q_rope (64)] of each row into TMEM (lanes 0-15, one
+    // row per lane), as bf16 pairs; lanes 16-31 store zeros into the O
+    // half-lanes, which the first PV overwrites.
     {
-      const bool load = lane < 16 && in_range && grow0 + row < p.rows;
-      const long long grow = grow0 + row;
+      const int row_q = 16 * qd + (lane & 15);
+      const bool load = lane < 16 && hb * kM + row_q < p.rows_unit && grow0 + row_q < p.rows;
+      const long long grow = grow0 + row_q;
       for (int c = 0; c < (int)kQCols / 32; ++c) {
         uint32_t v[32];
 #pragma unroll
@@ -257,11 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t0 = t_begin + j * kTk;
       if (ok) ok = ptx::mbar_wait(&s_full[sb], (j >> 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
-      uint32_t sv[kTk];
+      uint32_t sv[kTk / 2];                      // tokens 2 v + half, v = 0..31
       if (ok) {
         ptx::tc_fence_after();
-        ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * sb, sv);
-        ptx::tmem_ld32(tl + kSCol + (uint32_t)kTk * sb + 32u, sv + 32);
+        ptx::tmem_ld16x64(tl + kSCol + (uint32_t)kTk * sb, sv);
         ptx::tmem_ld_wait();
       }
       ptx::tc_fence_before();
@@ -269,14 +271,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) ptx::mbar_arrive(&s_free[sb]);
       float factor = 1.f;
       int need = 0;
-      if (lane < 16 && ok) {
+      if (ok) {
         float mx = -INFINITY;
 #pragma unroll
-        for (int t = 0; t < kTk; ++t) {
-          const float x = (t0 + t < vis) ? __uint_as_float(sv[t]) * p.scale_log2 : -INFINITY;
-          sv[t] = __float_as_uint(x);
+        for (int v = 0; v < kTk / 2; ++v) {
+          const float x = (t0 + 2 * v + half < vis) ? __uint_as_float(sv[v]) * p.scale_log2 : -INFINITY;
+          sv[v] = __float_as_uint(x);
           mx = fmaxf(mx, x);
         }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));   // the row's other half
         if (m_used == -INFINITY) {
           m_used = mx;                            // O holds only zeros so far
         } else if (mx > m_used + kRescaleLog2) {
@@ -287,17 +290,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float acc = 0.f;
 #pragma unroll
-        for (int t = 0; t < kTk; ++t) {
-          const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(__uint_as_float(sv[t]) - m_used);
-          sv[t] = __float_as_uint(e);
+        for (int v = 0; v < kTk / 2; ++v) {
+          const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(__uint_as_float(sv[v]) - m_used);
+          sv[v] = __float_as_uint(e);
           acc += e;
         }
-        l_sum += acc;
+        l_sum += acc;                            // this thread's half of the row sum
       } else {
 #pragma unroll
-        for (int t = 0; t < kTk; ++t) sv[t] = 0u;
+        for (int v = 0; v < kTk / 2; ++v) sv[v] = 0u;
       }
-      const float f_row = __shfl_sync(0xffffffffu, factor, o_dp);
+      const float f_row = factor;                // O rows use the same thread mapping
       const bool any_rescale = __any_sync(0xffffffffu, need) != 0;
       // PV(j-1) must be done before O is rescaled and before P is overwritten
       if (ok && j >= 1) ok = ptx::mbar_wait(&pv_done, (j - 1) & 1);
@@ -324,16 +327,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_uint4(0, 0, 0, 0);
         }
       }
-      if (lane < 16) {
+      {
+        // P row: the half == 0 thread writes tokens 0..31, its partner 32..63;
+        // each trades the 16 values the other one needs (one shuffle each)
+        uint32_t pk[kTk / 4];                    // bf16 pairs of tokens 32 half + 2 i, + 1
 #pragma unroll
-        for (int g8 = 0; g8 < kTk / 8; ++g8) {
-          uint4 v;
-          v.x = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 0]), __uint_as_float(sv[8 * g8 + 1]));
-          v.y = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 2]), __uint_as_float(sv[8 * g8 + 3]));
-          v.z = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 4]), __uint_as_float(sv[8 * g8 + 5]));
-          v.w = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 6]), __uint_as_float(sv[8 * g8 + 7]));
-          *reinterpret_cast<uint4*>(sP + ptx::swz128(row, g8)) = v;
+        for (int i = 0; i < kTk / 4; ++i) {
+          const uint32_t send = half ? sv[i] : sv[kTk / 4 + i];
+          const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 2);
+          pk[i] = half ? ptx::pack_bf16(__uint_as_float(recv), __uint_as_float(sv[kTk / 4 + i]))
+                       : ptx::pack_bf16(__uint_as_float(sv[i]), __uint_as_float(recv));
         }
+#pragma unroll
+        for (int g = 0; g < kTk / 16; ++g)
+          *reinterpret_cast<uint4*>(sP + ptx::swz128(row, 4 * half + g)) =
+              make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
@@ -350,11 +358,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the whole ring is idle now (every load was consumed): stage O there
     asm volatile("bar.sync 1, 128;" ::: "memory");
     float* stage = reinterpret_cast<float*>(sKV);
-    const float l_o = __shfl_sync(0xffffffffu, l_sum, o_dp);
-    const float inv_o = (l_o > 0.f && have_o) ? 1.f / l_o : 0.f;
+    const float l_row = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 2);
+    const float inv_o = (l_row > 0.f && have_o) ? 1.f / l_row : 0.f;
     if (have_o) {
       ptx::tc_fence_after();
-      const int orow = 16 * qd + o_dp, par = (lane >> 1) & 1;
+      const int orow = row, par = half;
       for (int c = 0; c < kR / 64; ++c) {
         uint32_t ov[32];
         ptx::tmem_ld16x64(tl + kOLane + 64u * c, ov);
@@ -372,9 +380,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float4 v = have_o ? *reinterpret_cast<const float4*>(stage + rr * kOStride + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
       *reinterpret_cast<float4*>(p.o_part + ((long long)split * p.rows + grow) * kR + c4) = v;
     }
-    if (in_range && ok && lane < 16) {
-      const bool empty = !(l_sum > 0.f) || !have_o;
-      const float lse = empty ? -INFINITY : (m_used + log2f(l_sum)) * 0.69314718055994531f;
+    if (in_range && ok && half == 0) {
+      const bool empty = !(l_row > 0.f) || !have_o;
+      const float lse = empty ? -INFINITY : (m_used + log2f(l_row)) * 0.69314718055994531f;
       p.lse[(long long)split * p.rows + grow0 + row] = lse;
     }
   }

@@ -179,13 +179,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ptx::tc_fence_after();
           const uint32_t a_addr = base + s * kStageBytes;
-          const uint32_t b_addr = a_addr + kABytes;
+          const uint64_t ad0 = ptx::umma_desc_sw128(a_addr, 16, 1024);
+          const uint64_t bd0 = ptx::umma_desc_sw128(a_addr + kABytes, kBBox, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kKC / 16; ++kk) {
-            const uint64_t ad = ptx::umma_desc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = ptx::umma_desc_sw128(b_addr + kk * 16 * 128, kBBox, 1024);
-            ptx::umma_bf16(d, ad, bd, idesc, (kc | kk) != 0);
-          }
+          for (int kk = 0; kk < kKC / 16; ++kk)
+            ptx::umma_bf16(d, ptx::umma_desc_add(ad0, kk * 32), ptx::umma_desc_add(bd0, kk * 16 * 128), idesc,
+                           (kc | kk) != 0);
           ptx::umma_commit(&empty_bar[s]);
         }
         if (!ok) break;

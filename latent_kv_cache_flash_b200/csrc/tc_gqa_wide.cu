@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------- QK issuer, TMEM owner
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = ptx::idesc_bf16(kM, kT, false, false);
-      const uint32_t q_addr = ptx::smem_u32(sQ), kv_addr = ptx::smem_u32(sKV);
+      const uint32_t kv_addr = ptx::smem_u32(sKV);
+      const uint64_t ad0 = ptx::umma_desc_sw128(ptx::smem_u32(sQ), 16, 1024);
       bool ok = ptx::mbar_wait(&q_full, 0);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kStages, sb = j & 1;
@@ -148,14 +149,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t st_addr = kv_addr + s * kStageBytes;
+        const uint64_t bd0 = ptx::umma_desc_sw128(kv_addr + s * kStageBytes, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kDqk / 16; ++kk) {
-          const uint32_t koff = kk >> 2, kin = (kk & 3) * 32;
-          const uint64_t a = ptx::umma_desc_sw128(q_addr + koff * kQChunkBytes + kin, 16, 1024);
-          const uint64_t bd = ptx::umma_desc_sw128(st_addr + koff * kChunkBytes + kin, 16, 1024);
-          ptx::umma_bf16(tmem + kSCol + (uint32_t)kT * sb, a, bd, idesc_qk, kk > 0);
-        }
+        for (int kk = 0; kk < kDqk / 16; ++kk)
+          ptx::umma_bf16(tmem + kSCol + (uint32_t)kT * sb,
+                         ptx::umma_desc_add(ad0, (kk >> 2) * kQChunkBytes + (kk & 3) * 32),
+                         ptx::umma_desc_add(bd0, (kk >> 2) * kChunkBytes + (kk & 3) * 32), idesc_qk, kk > 0);
         ptx::umma_commit(&s_full[sb]);
       }
       if (!ok) {
@@ -169,20 +168,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- PV issuer
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_pv = ptx::idesc_bf16(kM, kDv, false, true);
-      const uint32_t kv_addr = ptx::smem_u32(sKV), p_addr = ptx::smem_u32(sP);
+      const uint32_t kv_addr = ptx::smem_u32(sKV);
+      const uint64_t ad0 = ptx::umma_desc_sw128(ptx::smem_u32(sP), 16, 1024);
       bool ok = true;
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kStages;
         ok = ptx::mbar_wait(&p_full, j & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t v_addr = kv_addr + s * kStageBytes + kKChunks * kChunkBytes;
+        const uint64_t bd0 = ptx::umma_desc_sw128(kv_addr + s * kStageBytes + kKChunks * kChunkBytes, kChunkBytes, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kT / 16; ++kk) {
-          const uint64_t a = ptx::umma_desc_sw128(p_addr + kk * 32, 16, 1024);
-          const uint64_t bd = ptx::umma_desc_sw128(v_addr + kk * 16 * 128, kChunkBytes, 1024);
-          ptx::umma_bf16(tmem + kOCol, a, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kT / 16; ++kk)
+          ptx::umma_bf16(tmem + kOCol, ptx::umma_desc_add(ad0, kk * 32), ptx::umma_desc_add(bd0, kk * 16 * 128),
+                         idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         ptx::umma_commit(&pv_done);
         ptx::umma_commit(&kv_empty[s]);
       }
