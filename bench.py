@@ -52,7 +52,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
-    ap.add_argument("--sweep", choices=["crossover", "context", "ragged"],
+    ap.add_argument("--tp", action="store_true",
+                    help="with --gpus N > 1: split the groups of one batch over the ranks (strong scaling) "
+                         "instead of giving every rank its own batch")
+    ap.add_argument("--sweep", choices=["crossover", "context", "ragged", "capacity"],
                     help="instead of the headline line, time both decode paths over a workload sweep "
                          "(one JSON line per point)")
     return ap.parse_args()
@@ -248,9 +251,14 @@ def run_ours(args):
     hbm, tf_burst, tf_sust, peak_src = load_peaks()
 
     wl = workload(args.sq)
-    wl.seed = multi.rank_seed(wl.seed, rank)
-    d = wl.dims
+    tp = args.tp and world > 1
+    if not tp:
+        wl.seed = multi.rank_seed(wl.seed, rank)   # replicas: every rank its own batch
     inp = synth.make_inputs(wl, dev)
+    if tp:
+        inp = multi.tp_shard(inp, world, rank)    # the same batch; this rank's groups and heads
+        wl = inp.wl
+    d = wl.dims
     dims = gqla.make_dims(d)
     lay = gqla.make_layout(inp.seq_lens, inp.max_seq_len, 0, inp.capacity, None, 0)
     ks, vs = synth.expanded_pool_shapes(inp)
@@ -394,7 +402,8 @@ def run_ours(args):
 
     alg = algorithmic(wl)
     tokens = B * d.s_q
-    value = multi.job_tokens_per_s(tokens, 1, world, ms_step)
+    # replicas decode world batches per step; tensor-parallel ranks share one
+    value = multi.job_tokens_per_s(tokens, 1, 1 if tp else world, ms_step)
     # dominant kernel: the slower decode call of the step
     if ms_gqa >= ms_absorb:
         name, ms_dom, bytes_dom = "gqla_decode_gqa", ms_gqa, alg["gqa_bytes"]
@@ -427,7 +436,8 @@ def run_ours(args):
     d2h = out_host.numel() * out_host.element_size()
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if tp else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, random-init weights)",
         "config": {"workload": "%s B%d L%d s_q%d" % (wl.name, B, wl.seq_len, d.s_q), "batch": B,
                    "seq_len": wl.seq_len, "s_q": d.s_q, "n_h": d.n_h, "G": d.G, "d_nope": d.d_nope,
@@ -439,9 +449,12 @@ def run_ours(args):
                    "eager_ms_per_step": eager_ms,
                    "l2": "no flush: inputs larger than L2 (latent %.0f MB, expanded cache %.0f MB)" % (
                        alg["absorb_bytes"] / 1e6, alg["gqa_bytes"] / 1e6),
-                   "parallelism": "replicas x%d (batch-sharded, no collective)" % world},
+                   "parallelism": ("tp%d over groups (each rank: G/%d groups and their heads; no collective "
+                                   "inside attention)" % (world, world)) if tp else
+                                  "replicas x%d (batch-sharded, no collective)" % world},
         "roofline": roof,
-        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": (1 if tp else world) * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "clocks": clk,
@@ -546,12 +559,96 @@ def time_paths(inp, reps, hbm, tf_burst, expand=True):
     return res
 
 
+def capacity_point(d, L, budget_bytes, path, reps, hbm, tf_burst, max_batch=4096):
+    """Largest batch of L-token sequences whose cache for this path fits in
+    budget_bytes, and one decode call's device time at that batch.  Only the
+    path's own cache is allocated (filled with seeded random bf16: decode time
+    does not depend on the values)."""
+    import torch
+    from latent_kv_cache_flash_b200 import gqla, synth
+    dev = torch.device("cuda")
+    dd = dataclasses.replace(d, k_shared_rope=(path == "gqa_shared_rope"))
+    dims = gqla.make_dims(dd)
+    per_token = gqla.gqla_cache_bytes_per_token(dims, gqla.GQLA_PATH_ABSORB if path == "absorb" else gqla.GQLA_PATH_GQA)
+    B = min(max_batch, int(budget_bytes // (per_token * L)))
+    if B < 1:
+        return {"batch": 0}
+    g = torch.Generator(device=dev)
+    g.manual_seed(2)
+    lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    lay = gqla.make_layout(lens, L, 0, L)
+    q = synth._randn_chunked((B, d.s_q, d.n_h, d.d_qk), g, dev, d.torch_dtype)
+    out = torch.empty((B, d.s_q, d.n_h, d.d_v), dtype=d.torch_dtype, device=dev)
+    lse = torch.empty((B, d.s_q, d.n_h), device=dev)
+    keys = B * sum(L - d.s_q + i + 1 for i in range(d.s_q))
+    if path == "absorb":
+        latent = synth._randn_chunked((B, L, d.r + d.d_rope), g, dev, d.torch_dtype)
+        W_uk = synth._randn_chunked((d.G, d.r, d.d_nope), g, dev, d.torch_dtype)
+        W_uv = synth._randn_chunked((d.G, d.r, d.d_v), g, dev, d.torch_dtype)
+        ws = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_ABSORB, dev)
+        fn = lambda: gqla.gqla_decode_absorb(dims, lay, q, latent, W_uk, W_uv, out, lse, 0, ws)
+        flops = d.n_h * keys * 2 * (2 * d.r + d.d_rope)
+        pools = (latent,)
+    else:
+        kw = d.G * d.d_nope + d.d_rope if dd.k_shared_rope else d.G * d.d_qk
+        kp = synth._randn_chunked((B, L, kw), g, dev, d.torch_dtype)
+        vp = synth._randn_chunked((B, L, d.G * d.d_v), g, dev, d.torch_dtype)
+        ws = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_GQA, dev)
+        fn = lambda: gqla.gqla_decode_gqa(dims, lay, q, kp, vp, out, lse, 0, ws)
+        flops = d.n_h * keys * 2 * (d.d_qk + d.d_v)
+        pools = (kp, vp)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = per_token * L * B
+    t_roof = max(nbytes / (hbm * 1e9), flops / (tf_burst * 1e12))
+    del pools
+    return {"batch": B, "cache_bytes": nbytes, "ms": ms, "tokens_per_s": B * d.s_q / (ms * 1e-3),
+            "roofline_frac": t_roof / (ms * 1e-3)}
+
+
+def run_capacity(args):
+    """Capacity-tuned comparison: under one cache budget per GPU for this
+    layer, each path decodes the largest batch that fits.  The DeepSeek-V3
+    layer whole on one GPU, and one rank's share of it under 8-way group
+    tensor parallelism (16 heads, 2 groups; the absorb path keeps the whole
+    latent cache on every rank)."""
+    import torch
+    from latent_kv_cache_flash_b200 import build, synth
+    build.build()
+    hbm, tf_burst, _, _ = load_peaks()
+    budget = 16 * 2 ** 30
+    layers = [("DeepSeek-V3 layer, one GPU", synth.Dims(n_h=128, G=16, d_nope=128, d_rope=64, d_v=128, r=512)),
+              ("DeepSeek-V3 layer, one rank of 8-way group TP",
+               synth.Dims(n_h=16, G=2, d_nope=128, d_rope=64, d_v=128, r=512))]
+    for name, d in layers:
+        for L in (8192, 32768):
+            line = {"sweep": "capacity", "layer": name, "n_h": d.n_h, "G": d.G, "s_q": d.s_q, "seq_len": L,
+                    "budget_bytes": budget}
+            for path in ("absorb", "gqa", "gqa_shared_rope"):
+                line[path] = capacity_point(d, L, budget, path, max(5, args.steps // 10), hbm, tf_burst)
+                torch.cuda.empty_cache()
+            ok = {k: v for k, v in line.items() if isinstance(v, dict) and v.get("batch")}
+            line["fastest_at_capacity"] = max(ok, key=lambda k: ok[k]["tokens_per_s"])
+            print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_sweep(args):
     """Both decode paths over the crossover, context or ragged workloads."""
     import torch
     from latent_kv_cache_flash_b200 import build, synth
     build.build()
     hbm, tf_burst, _, _ = load_peaks()
+    if args.sweep == "capacity":
+        return run_capacity(args)
     if args.sweep == "crossover":
         points = [synth.crossover(G, s_q) for G in (1, 2, 4, 8, 16, 32, 128) for s_q in (1, 2, 4)]
     elif args.sweep == "context":
