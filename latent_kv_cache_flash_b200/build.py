@@ -73,7 +73,9 @@ def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False)
                 sys.stderr.write("nvcc failed on %s\n" % src)
     if failed:
         raise RuntimeError("CUDA build failed")
-    relink = jobs or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs)
+    # a source added or removed changes the directory's mtime: relink then too
+    relink = jobs or not os.path.exists(LIB) or os.path.getmtime(CSRC) > os.path.getmtime(LIB) or \
+        any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs)
     if relink:
         tmp = LIB + ".tmp"
         cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcuda"]

@@ -281,3 +281,49 @@ def test_gqa_many_rows_per_group_paged(G, s_q, splits):
     inp = _wl(d, 3, [777, 1500, 64], page=64, seed=40 + G)
     out, lse = H.run_decode(inp, "gqa", num_splits=splits)
     H.check_units(inp, out, lse, H.sample_units(inp, 5, seed=G), "gqa wide G=%d s_q=%d S=%d" % (G, s_q, splits))
+
+
+# ---- absorb at 128 heads: several 64-row blocks per sequence -------------------
+@pytest.mark.parametrize("s_q,splits", [(1, 0), (1, 4), (2, 3), (4, 0)])
+def test_absorb_128_heads_paged_ragged_edges(s_q, splits):
+    """n_h = 128 (2 to 8 row blocks a sequence): paged, ragged, with
+    page-boundary and tiny lengths (L = s_q, one page, one token past a page),
+    every unit against the oracle."""
+    d = synth.Dims(**DSV3, s_q=s_q)
+    lens = [s_q, 64, 65, 1313, 2048]
+    inp = _wl(d, len(lens), lens, page=64, seed=90 + s_q)
+    out, lse = H.run_decode(inp, "absorb", num_splits=splits)
+    H.check_units(inp, out, lse, H.all_units(inp), "absorb 128 heads s_q=%d S=%d" % (s_q, splits))
+
+
+@pytest.mark.parametrize("peak", [1.0, 3.0])
+def test_absorb_128_heads_growing_scores(peak):
+    """Scores that rise along the sequence force the lazy rescale in every row
+    block; contiguous cache, n_h = 128, s_q = 2."""
+    d = synth.Dims(**DSV3, s_q=2)
+    lens = [1500, 700]
+    inp = _wl(d, 2, lens, seed=23)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(6)
+    u = torch.randn(d.d_rope, generator=g, device=DEV) * peak
+    q = inp.q.float()
+    q[..., d.d_nope:] = u + 0.05 * torch.randn(q[..., d.d_nope:].shape, generator=g, device=DEV)
+    inp.q.copy_(q.to(inp.q.dtype))
+    for b, L in enumerate(lens):
+        rows = inp.latent[b].float()
+        t = torch.arange(rows.shape[0], device=DEV, dtype=torch.float32)[:, None]
+        rows[:, d.r:] = 0.1 * rows[:, d.r:] + (4.0 * t / L) * u[None, :] / peak
+        inp.latent[b] = rows.to(inp.latent.dtype)
+    for splits in (1, 0):
+        out, lse = H.run_decode(inp, "absorb", num_splits=splits)
+        H.check_units(inp, out, lse, H.all_units(inp), "absorb 128 heads growing peak=%g S=%d" % (peak, splits))
+
+
+def test_absorb_128_heads_matches_gqa_full_tensor():
+    """Absorb and GQA on the same weights at n_h = 128, whole tensors."""
+    d = synth.Dims(**DSV3, s_q=1)
+    inp = _wl(d, 4, [3000, 1, 777, 4096], page=64, seed=95)
+    a_o, a_l = H.run_decode(inp, "absorb")
+    g_o, g_l = H.run_decode(inp, "gqa")
+    H.assert_close(a_o.float().cpu().numpy(), g_o.float().cpu().numpy(), "bf16", "absorb vs gqa out")
+    H.assert_close(a_l.cpu().numpy(), g_l.cpu().numpy(), "bf16", "absorb vs gqa lse")
