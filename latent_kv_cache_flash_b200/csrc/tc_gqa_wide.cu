@@ -8,16 +8,23 @@
 // on the 5th-generation tensor cores with the rows as the MMA's M.
 //
 // One CTA per (key-range split, sequence, group, block of 128 rows):
-//  * the 128 x 192 query tile is gathered into 128-byte-swizzled shared
-//    memory once; 64-token K (64 x 192) and V (64 x 128) tiles stream in with
-//    TMA (2-D maps over the pools' token rows; a group's chunks are column
-//    offsets) into a 4-stage mbarrier ring;
-//  * warp 1 issues S = Q K^T (12 tcgen05.mma, M=128, N=64, K=16) into a
-//    double-buffered S in TMEM; warp 6 issues O += P V (4 tcgen05.mma,
-//    M=128, N=128, K=16, V as an MN-major operand) into O in TMEM;
-//  * warps 2-5 own one row each: online softmax in the log2 domain with lazy
-//    rescaling of O (only when a row maximum grows by more than 2^8), P to
-//    shared memory, and the normalised output and log-sum-exp at the end.
+//  * the 128 x 192 query tile is stored into TMEM once (the A operand of
+//    the score MMAs), which leaves shared memory to a 4-stage mbarrier ring
+//    of 64-token K (64 x 192) and V (64 x 128) tiles (TMA, 2-D maps over the
+//    pools' token rows; a group's chunks are column offsets) and two P tiles;
+//  * warp 1 issues S = Q K^T (12 tcgen05.mma, M=128, N=64, K=16) into S[j % 2]
+//    in TMEM; warp 6 issues O[j % 2] += P[j % 2] V (4 tcgen05.mma, M=128,
+//    N=128, K=16, V as an MN-major operand);
+//  * two softmax warpgroups take alternate tiles (warps 2-5 the even ones,
+//    8-11 the odd ones), each with its own running maximum, sum and O
+//    accumulator: the softmax of 128 rows x 64 tokens takes about twice the
+//    tensor pipe's time for the tile, so one warpgroup would leave the pipe
+//    idle half the time.  Within a group a thread owns one row: online
+//    softmax in the log2 domain with lazy rescaling of its O (only when the
+//    row maximum grows by more than 2^8), P to shared memory;
+//  * at the end the even group merges the two states (the odd group's
+//    maximum and sum through shared memory, both O halves straight from
+//    TMEM) and writes the normalised output and the log-sum-exp.
 #include <math.h>
 
 #include "ptx.cuh"
@@ -36,13 +43,11 @@ constexpr int kKChunks = kDqk / 64;           // 3 K chunks of 64 dims
 constexpr int kVChunks = kDv / 64;            // 2 V chunks
 constexpr int kChunkBytes = kT * 128;         // 8 KB
 constexpr int kStageBytes = (kKChunks + kVChunks) * kChunkBytes;   // 40 KB
-constexpr int kQChunkBytes = kM * 128;        // 16 KB
-constexpr int kQBytes = kKChunks * kQChunkBytes;                     // 48 KB
 constexpr int kPBytes = kM * 128;             // 128 rows x 64 tokens (bf16)
-constexpr size_t kSmemBytes = (size_t)kQBytes + (size_t)kStages * kStageBytes + kPBytes + 1024;
-constexpr uint32_t kTmemCols = 256;           // S: 2 x 64, O: 128
-constexpr uint32_t kSCol = 0, kOCol = 128;
-constexpr int kThreads = 7 * 32;
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 2 * kPBytes + 2 * kM * 4 + 1024;
+constexpr uint32_t kTmemCols = 512;           // S: 2 x 64 at 0, O: 2 x 128 at 128, Q: 96 at 384
+constexpr uint32_t kSCol = 0, kOCol = 128, kQCol = 384;
+constexpr int kThreads = 12 * 32;
 constexpr float kRescaleLog2 = 8.f;
 
 struct WideParams {
@@ -66,11 +71,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const WideParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + kQBytes;
-  uint8_t* sP = sKV + kStages * kStageBytes;
-  __shared__ __align__(8) uint64_t q_full, p_full, pv_done, qk_drain, pv_drain;
-  __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2];
+  uint8_t* sKV = smem;
+  uint8_t* sP = sKV + kStages * kStageBytes;           // P[2]: one per softmax group
+  float* sML = reinterpret_cast<float*>(sP + 2 * kPBytes);   // the odd group's row max and sum
+  __shared__ __align__(8) uint64_t q_full, qk_drain, pv_drain;
+  __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], p_full[2],
+      pv_done[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -81,8 +87,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&q_full, 4);
-    ptx::mbar_init(&p_full, 4);
-    ptx::mbar_init(&pv_done, 1);
     ptx::mbar_init(&qk_drain, 1);
     ptx::mbar_init(&pv_drain, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -92,6 +96,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&s_full[s], 1);
       ptx::mbar_init(&s_free[s], 4);
+      ptx::mbar_init(&p_full[s], 4);
+      ptx::mbar_init(&pv_done[s], 1);
     }
     abort_flag = 0;
     ptx::fence_barrier_init();
@@ -141,8 +147,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = ptx::idesc_bf16(kM, kT, false, false);
       const uint32_t kv_addr = ptx::smem_u32(sKV);
-      const uint64_t ad0 = ptx::umma_desc_sw128(ptx::smem_u32(sQ), 16, 1024);
       bool ok = ptx::mbar_wait(&q_full, 0);
+      ptx::tc_fence_after();
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kStages, sb = j & 1;
         ok = ptx::mbar_wait(&kv_full[s], (j / kStages) & 1);
@@ -152,9 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bd0 = ptx::umma_desc_sw128(kv_addr + s * kStageBytes, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < kDqk / 16; ++kk)
-          ptx::umma_bf16(tmem + kSCol + (uint32_t)kT * sb,
-                         ptx::umma_desc_add(ad0, (kk >> 2) * kQChunkBytes + (kk & 3) * 32),
-                         ptx::umma_desc_add(bd0, (kk >> 2) * kChunkBytes + (kk & 3) * 32), idesc_qk, kk > 0);
+          ptx::umma_bf16_ts(tmem + kSCol + (uint32_t)kT * sb, tmem + kQCol + 8u * kk,
+                            ptx::umma_desc_add(bd0, (kk >> 2) * kChunkBytes + (kk & 3) * 32), idesc_qk, kk > 0);
         ptx::umma_commit(&s_full[sb]);
       }
       if (!ok) {
@@ -172,16 +177,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t ad0 = ptx::umma_desc_sw128(ptx::smem_u32(sP), 16, 1024);
       bool ok = true;
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kStages;
-        ok = ptx::mbar_wait(&p_full, j & 1);
+        const int s = j % kStages, sb = j & 1;
+        ok = ptx::mbar_wait(&p_full[sb], (j >> 1) & 1);
         if (!ok) break;
         ptx::tc_fence_after();
         const uint64_t bd0 = ptx::umma_desc_sw128(kv_addr + s * kStageBytes + kKChunks * kChunkBytes, kChunkBytes, 1024);
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
-          ptx::umma_bf16(tmem + kOCol, ptx::umma_desc_add(ad0, kk * 32), ptx::umma_desc_add(bd0, kk * 16 * 128),
-                         idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        ptx::umma_commit(&pv_done);
+          ptx::umma_bf16(tmem + kOCol + (uint32_t)kDv * sb, ptx::umma_desc_add(ad0, sb * kPBytes + kk * 32),
+                         ptx::umma_desc_add(bd0, kk * 16 * 128), idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
+        ptx::umma_commit(&pv_done[sb]);
         ptx::umma_commit(&kv_empty[s]);
       }
       if (!ok) {
@@ -191,95 +196,125 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::umma_commit(&pv_drain);
       ptx::mbar_wait(&pv_drain, 0);
     }
-  } else {
-    // ------------------------------------------- softmax + epilogue warps
+  } else if (warp >= 2 && warp != 6 && warp != 7) {
+    // ----------------------------------- softmax warpgroups and epilogue
+    const int gp = warp >= 8 ? 1 : 0;           // this group's tiles: j % 2 == gp
     const int qd = warp & 3;
     const int row = 32 * qd + lane;             // M row = TMEM lane
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+    const uint32_t o_col = kOCol + (uint32_t)kDv * gp;
+    uint8_t* sPg = sP + gp * kPBytes;
     const int r_local = rb * kM + row;
     const bool in_range = r_local < p.rows_unit;
     const bool valid = in_range && L >= 0;
     const int i_q = in_range ? r_local / p.m : 0;
     const long long grow = in_range ? ((long long)b * p.s_q + i_q) * p.n_h + g * p.m + r_local % p.m : 0;
     const int vis = valid ? L - p.s_q + i_q + 1 : 0;
-    // this row's query into the swizzled Q tile (zeros for padding rows)
-    for (int c = 0; c < kKChunks; ++c) {
+    if (gp == 0) {
+      // this row's query into TMEM (lane = row, bf16 pairs; zeros for padding rows)
+      for (int c = 0; c < kKChunks; ++c) {
+        uint32_t v[32];
 #pragma unroll
-      for (int gi = 0; gi < 8; ++gi) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (in_range) v = *reinterpret_cast<const uint4*>(p.q + grow * kDqk + 64 * c + 8 * gi);
-        *reinterpret_cast<uint4*>(sQ + c * kQChunkBytes + ptx::swz128(row, gi)) = v;
+        for (int e = 0; e < 32; e += 4) {
+          uint4 w = make_uint4(0, 0, 0, 0);
+          if (in_range) w = *reinterpret_cast<const uint4*>(p.q + grow * kDqk + 64 * c + 2 * e);
+          v[e] = w.x;
+          v[e + 1] = w.y;
+          v[e + 2] = w.z;
+          v[e + 3] = w.w;
+        }
+        ptx::tmem_st32(tl + kQCol + 32u * c, v);
       }
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&q_full);
     }
-    ptx::fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&q_full);
 
     float m_used = -INFINITY, l_sum = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int sb = j & 1, s = j % kStages;
+    int last = -1;                               // this group's last tile
+    for (int j = gp; j < n_tiles; j += 2) {
+      const int s = j % kStages;
       const int t0 = t_begin + j * kT;
-      if (ok) ok = ptx::mbar_wait(&s_full[sb], (j >> 1) & 1);
+      last = j;
+      if (ok) ok = ptx::mbar_wait(&s_full[gp], (j >> 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
-      uint32_t sv[kT];
+      // the row maximum over the tile's 64 scores, read in two halves; S[gp]
+      // is next written for tile j + 2, this group's own next tile
+      float mx = -INFINITY;
       if (ok) {
         ptx::tc_fence_after();
-        ptx::tmem_ld32(tl + kSCol + (uint32_t)kT * sb, sv);
-        ptx::tmem_ld32(tl + kSCol + (uint32_t)kT * sb + 32u, sv + 32);
-        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sv[32];
+          ptx::tmem_ld32(tl + kSCol + (uint32_t)kT * gp + 32u * h, sv);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            if (t0 + 32 * h + t < vis) mx = fmaxf(mx, __uint_as_float(sv[t]) * p.scale_log2);
+        }
       }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s_free[sb]);
       float factor = 1.f;
       int need = 0;
-      if (ok) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int t = 0; t < kT; ++t) {
-          const float x = (t0 + t < vis) ? __uint_as_float(sv[t]) * p.scale_log2 : -INFINITY;
-          sv[t] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-        if (m_used == -INFINITY) {
-          m_used = mx;
-        } else if (mx > m_used + kRescaleLog2) {
-          factor = ptx::fast_exp2(m_used - mx);
-          need = 1;
-          l_sum *= factor;
-          m_used = mx;
-        }
-        float acc = 0.f;
-#pragma unroll
-        for (int t = 0; t < kT; ++t) {
-          const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(__uint_as_float(sv[t]) - m_used);
-          sv[t] = __float_as_uint(e);
-          acc += e;
-        }
-        l_sum += acc;
-      } else {
-#pragma unroll
-        for (int t = 0; t < kT; ++t) sv[t] = 0u;
+      if (m_used == -INFINITY) {
+        m_used = mx;                              // this group's O holds only zeros so far
+      } else if (mx > m_used + kRescaleLog2) {
+        factor = ptx::fast_exp2(m_used - mx);
+        need = 1;
+        l_sum *= factor;
+        m_used = mx;
       }
       const bool any_rescale = __any_sync(0xffffffffu, need) != 0;
-      if (ok && j >= 1) ok = ptx::mbar_wait(&pv_done, (j - 1) & 1);
+      // this group's previous PV (tile j - 2) must be done before its O is
+      // rescaled and its P overwritten
+      if (ok && j >= 2) ok = ptx::mbar_wait(&pv_done[gp], ((j >> 1) - 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (ok && any_rescale) {
         ptx::tc_fence_after();
         for (int c = 0; c < kDv / 32; ++c) {
           uint32_t ov[32];
-          ptx::tmem_ld32(tl + kOCol + 32u * c, ov);
+          ptx::tmem_ld32(tl + o_col + 32u * c, ov);
           ptx::tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
-          ptx::tmem_st32(tl + kOCol + 32u * c, ov);
+          ptx::tmem_st32(tl + o_col + 32u * c, ov);
         }
         ptx::tmem_st_wait();
       }
+      // P = 2^(s - m) in bf16, the two halves read again from TMEM
+      float acc = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sv[32];
+        if (ok) {
+          ptx::tmem_ld32(tl + kSCol + (uint32_t)kT * gp + 32u * h, sv);
+          ptx::tmem_ld_wait();
+        }
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          const float x = (ok && t0 + 32 * h + t < vis) ? __uint_as_float(sv[t]) * p.scale_log2 : -INFINITY;
+          const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(x - m_used);
+          sv[t] = __float_as_uint(e);
+          acc += e;
+        }
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+          uint4 v;
+          v.x = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 0]), __uint_as_float(sv[8 * g8 + 1]));
+          v.y = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 2]), __uint_as_float(sv[8 * g8 + 3]));
+          v.z = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 4]), __uint_as_float(sv[8 * g8 + 5]));
+          v.w = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 6]), __uint_as_float(sv[8 * g8 + 7]));
+          *reinterpret_cast<uint4*>(sPg + ptx::swz128(row, 4 * h + g8)) = v;
+        }
+      }
+      l_sum += acc;
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s_free[gp]);
       if (t0 + kT > L) {
         // value rows past the sequence may hold anything: zero them for PV
-        const int tid = threadIdx.x - 64;
+        const int tid = 32 * qd + lane;
         for (int idx = tid; idx < kT * kVChunks * 8; idx += 128) {
           const int tok = idx / (kVChunks * 8), rem = idx % (kVChunks * 8);
           if (t0 + tok >= L)
@@ -287,62 +322,72 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       ptx::swz128(tok, rem % 8)) = make_uint4(0, 0, 0, 0);
         }
       }
-#pragma unroll
-      for (int g8 = 0; g8 < kT / 8; ++g8) {
-        uint4 v;
-        v.x = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 0]), __uint_as_float(sv[8 * g8 + 1]));
-        v.y = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 2]), __uint_as_float(sv[8 * g8 + 3]));
-        v.z = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 4]), __uint_as_float(sv[8 * g8 + 5]));
-        v.w = ptx::pack_bf16(__uint_as_float(sv[8 * g8 + 6]), __uint_as_float(sv[8 * g8 + 7]));
-        *reinterpret_cast<uint4*>(sP + ptx::swz128(row, g8)) = v;
-      }
       ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (lane == 0) ptx::mbar_arrive(&p_full);
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + gp) : "memory");   // the tail zeroing is shared by the group
+      if (lane == 0) ptx::mbar_arrive(&p_full[gp]);
     }
     if (!ok && lane == 0) {
       flag_status(p.st, GQLA_DEV_TIMEOUT);
       atomicExch(&abort_flag, 1);
     }
     // ----------------------------------------------------------- epilogue
-    bool have_o = ok && n_tiles > 0 && ptx::mbar_wait(&pv_done, (n_tiles - 1) & 1);
+    bool have_o = ok && last >= 0 && ptx::mbar_wait(&pv_done[gp], (last >> 1) & 1);
     have_o = __all_sync(0xffffffffu, have_o);
-    ptx::tc_fence_after();
-    const bool empty = !(l_sum > 0.f) || !have_o;
-    const float inv = empty ? 0.f : 1.f / l_sum;
-    for (int c = 0; c < kDv / 32; ++c) {
-      uint32_t ov[32];
-      if (have_o) {
-        ptx::tmem_ld32(tl + kOCol + 32u * c, ov);
-        ptx::tmem_ld_wait();
-      }
-      if (in_range && ok) {
-        if (p.o_part) {
-          float* dst = p.o_part + ((long long)split * p.rows + grow) * kDv + 32 * c;
+    if (gp == 1) {
+      sML[row] = have_o ? m_used : -INFINITY;
+      sML[kM + row] = have_o ? l_sum : 0.f;
+    }
+    // both groups meet: the odd group's state is in shared memory and its O final
+    asm volatile("bar.sync 3, 256;" ::: "memory");
+    const bool ok1 = ok && *(volatile int*)&abort_flag == 0;   // a failed wait anywhere: write nothing
+    if (gp == 0) {
+      const float m1 = sML[row], l1 = sML[kM + row];
+      const bool have1 = m1 != -INFINITY;
+      const float m0 = have_o ? m_used : -INFINITY;
+      const float mt = fmaxf(m0, m1);
+      const float w0 = (m0 == -INFINITY) ? 0.f : ptx::fast_exp2(m0 - mt);
+      const float w1 = have1 ? ptx::fast_exp2(m1 - mt) : 0.f;
+      const float l = (have_o ? l_sum * w0 : 0.f) + (have1 ? l1 * w1 : 0.f);
+      const bool empty = !(l > 0.f) || !ok1;
+      const float inv = empty ? 0.f : 1.f / l;
+      const float a0 = w0 * inv, a1 = w1 * inv;
+      ptx::tc_fence_after();
+      for (int c = 0; c < kDv / 32; ++c) {
+        uint32_t o0[32], o1[32];
+        if (have_o) {
+          ptx::tmem_ld32(tl + kOCol + 32u * c, o0);
+          ptx::tmem_ld_wait();
+        }
+        if (__any_sync(0xffffffffu, have1)) {
+          ptx::tmem_ld32(tl + kOCol + (uint32_t)kDv + 32u * c, o1);
+          ptx::tmem_ld_wait();
+        }
+        float v[32];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + e) =
-                empty ? make_float4(0.f, 0.f, 0.f, 0.f)
-                      : make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
-                                    __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
-        } else {
-          __nv_bfloat16* dst = p.out + grow * kDv + 32 * c;
+        for (int e = 0; e < 32; ++e) {
+          float x = have_o ? __uint_as_float(o0[e]) * a0 : 0.f;
+          if (have1) x += __uint_as_float(o1[e]) * a1;   // select: an unused O half may hold anything
+          v[e] = empty ? 0.f : x;
+        }
+        if (in_range && ok1) {
+          if (p.o_part) {
+            float* dst = p.o_part + ((long long)split * p.rows + grow) * kDv + 32 * c;
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 w;
-            w.x = ptx::pack_bf16(empty ? 0.f : __uint_as_float(ov[e]) * inv, empty ? 0.f : __uint_as_float(ov[e + 1]) * inv);
-            w.y = ptx::pack_bf16(empty ? 0.f : __uint_as_float(ov[e + 2]) * inv, empty ? 0.f : __uint_as_float(ov[e + 3]) * inv);
-            w.z = ptx::pack_bf16(empty ? 0.f : __uint_as_float(ov[e + 4]) * inv, empty ? 0.f : __uint_as_float(ov[e + 5]) * inv);
-            w.w = ptx::pack_bf16(empty ? 0.f : __uint_as_float(ov[e + 6]) * inv, empty ? 0.f : __uint_as_float(ov[e + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + e) = w;
+            for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          } else {
+            __nv_bfloat16* dst = p.out + grow * kDv + 32 * c;
+#pragma unroll
+            for (int e = 0; e < 32; e += 8)
+              *reinterpret_cast<uint4*>(dst + e) =
+                  make_uint4(ptx::pack_bf16(v[e], v[e + 1]), ptx::pack_bf16(v[e + 2], v[e + 3]),
+                             ptx::pack_bf16(v[e + 4], v[e + 5]), ptx::pack_bf16(v[e + 6], v[e + 7]));
           }
         }
       }
-    }
-    if (in_range && ok && p.lse) {
-      const float lse = empty ? -INFINITY : (m_used + log2f(l_sum)) * 0.69314718055994531f;
-      p.lse[p.o_part ? (long long)split * p.rows + grow : grow] = lse;
+      if (in_range && ok1 && p.lse) {
+        const float lse = empty ? -INFINITY : (mt + log2f(l)) * 0.69314718055994531f;
+        p.lse[p.o_part ? (long long)split * p.rows + grow : grow] = lse;
+      }
     }
   }
   ptx::tc_fence_before();

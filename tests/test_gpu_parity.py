@@ -327,3 +327,26 @@ def test_absorb_128_heads_matches_gqa_full_tensor():
     g_o, g_l = H.run_decode(inp, "gqa")
     H.assert_close(a_o.float().cpu().numpy(), g_o.float().cpu().numpy(), "bf16", "absorb vs gqa out")
     H.assert_close(a_l.cpu().numpy(), g_l.cpu().numpy(), "bf16", "absorb vs gqa lse")
+
+
+@pytest.mark.parametrize("G,s_q,splits", [(1, 2, 1), (2, 4, 0), (2, 2, 3)])
+def test_gqa_wide_growing_scores(G, s_q, splits):
+    """The tcgen05 GQA kernel (m * s_q >= 64 rows a group) with scores that
+    rise along the sequence: both softmax warpgroups rescale their own
+    accumulator, and their states merge at the end."""
+    d = synth.Dims(n_h=128, G=G, d_nope=128, d_rope=64, d_v=128, r=512, s_q=s_q)
+    lens = [1500, 193]
+    inp = _wl(d, 2, lens, seed=31 + G)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(7)
+    u = torch.randn(d.d_rope, generator=g, device=DEV) * 2.0
+    q = inp.q.float()
+    q[..., d.d_nope:] = u + 0.05 * torch.randn(q[..., d.d_nope:].shape, generator=g, device=DEV)
+    inp.q.copy_(q.to(inp.q.dtype))
+    for b, L in enumerate(lens):
+        rows = inp.latent[b].float()
+        t = torch.arange(rows.shape[0], device=DEV, dtype=torch.float32)[:, None]
+        rows[:, d.r:] = 0.1 * rows[:, d.r:] + (4.0 * t / L) * u[None, :] / 2.0
+        inp.latent[b] = rows.to(inp.latent.dtype)
+    out, lse = H.run_decode(inp, "gqa", num_splits=splits)
+    H.check_units(inp, out, lse, H.all_units(inp), "gqa wide growing G=%d s_q=%d S=%d" % (G, s_q, splits))
