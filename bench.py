@@ -276,7 +276,12 @@ def run_ours(args):
         ws_a = ws_a0
     del ws_a0
     absorb_splits = [0]            # 0 = the library's plan for the whole GPU
-    ws_g = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_GQA, dev)
+    gqa_splits = [0]
+    ws_g = gqla.workspace_for(dims, lay, 8, gqla.GQLA_PATH_GQA, dev)
+    ws_g0 = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_GQA, dev)
+    if ws_g0.numel() > ws_g.numel():
+        ws_g = ws_g0
+    del ws_g0
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -299,7 +304,7 @@ def run_ours(args):
                                 ws_a, status)
 
     def gqa():
-        gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out_g, lse_g, 0, ws_g, status)
+        gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out_g, lse_g, gqa_splits[0], ws_g, status)
 
     def step():
         append_latent()
@@ -368,24 +373,25 @@ def run_ours(args):
             return g
 
         # The split plan of a call assumes it has the whole GPU; in the
-        # overlapped step the absorb call shares it with the GQA call, so its
-        # split count is tuned here: each candidate's graph is timed (untimed
-        # for the result) and the fastest is kept.
+        # overlapped step the two decode calls share it, so their split counts
+        # are tuned here: each candidate pair's graph is timed (outside the
+        # reported region) and the fastest pair is kept.
         tuned = {}
-        for cand in (0, 1, 2, 4, 8):
-            absorb_splits[0] = cand
-            g = capture()
-            tuned[cand] = timed(g.replay, 30) / 30
-            del g
-        absorb_splits[0] = min(tuned, key=tuned.get)
+        for ca in (0, 1, 2, 4):
+            for cg in (0, 2, 4, 8):
+                absorb_splits[0], gqa_splits[0] = ca, cg
+                g = capture()
+                tuned[(ca, cg)] = timed(g.replay, 30) / 30
+                del g
+        absorb_splits[0], gqa_splits[0] = min(tuned, key=tuned.get)
         graph = capture()
         ms_step = timed(graph.replay, args.steps) / args.steps
     else:
         ms_step = eager_ms
     # per-call breakdown (each over at least ~0.3 s of device time)
     reps = args.steps if args.no_clocks else max(args.steps, int(300.0 / max(ms_step, 1e-3)))
-    step_splits = absorb_splits[0]
-    absorb_splits[0] = 0                 # alone, the absorb call takes the library's own plan
+    step_splits = (absorb_splits[0], gqa_splits[0])
+    absorb_splits[0] = gqa_splits[0] = 0   # alone, each call takes the library's own plan
     ms_absorb = timed(absorb, reps) / reps
     ms_gqa = timed(gqa, reps) / reps
     ms_tail = timed(expand_tail, reps) / reps
@@ -415,7 +421,7 @@ def run_ours(args):
         out_host[0].copy_(out_a, non_blocking=True)
         out_host[1].copy_(out_g, non_blocking=True)
 
-    absorb_splits[0] = step_splits
+    absorb_splits[0], gqa_splits[0] = step_splits
     # the copies and the step's calls recorded once as a CUDA graph (the copies
     # read and write the pinned host buffers on every replay), then one replay
     # and a host wait per step
@@ -511,9 +517,11 @@ def run_ours(args):
                                         "hbm_gbs": exp_bytes / (ms_expand_full * 1e-3) / 1e9,
                                         "tc_frac": exp_flops / (ms_expand_full * 1e-3) / (tf_burst * 1e12)}},
         "splits": {"absorb": gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_ABSORB),
-                   "absorb_in_overlapped_step": gqla.gqla_num_splits(dims, lay, absorb_splits[0],
-                                                                     gqla.GQLA_PATH_ABSORB),
-                   "absorb_step_tuning_ms": ({str(k): v for k, v in tuned.items()} if tuned else None),
+                   "in_overlapped_step": {
+                       "absorb": gqla.gqla_num_splits(dims, lay, absorb_splits[0], gqla.GQLA_PATH_ABSORB),
+                       "gqa": gqla.gqla_num_splits(dims, lay, gqa_splits[0], gqla.GQLA_PATH_GQA)},
+                   "step_tuning_ms": ({"absorb %s, gqa %s" % (k[0] or "plan", k[1] or "plan"): v
+                                       for k, v in tuned.items()} if tuned else None),
                    "gqa": gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_GQA)},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

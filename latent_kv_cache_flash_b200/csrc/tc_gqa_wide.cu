@@ -291,6 +291,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_ld32(tl + kSCol + (uint32_t)kT * gp + 32u * h, sv);
           ptx::tmem_ld_wait();
         }
+        if (h == 1) {
+          // S[gp] is read for the last time: the next score MMAs may overwrite it
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&s_free[gp]);
+        }
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
           const float x = (ok && t0 + 32 * h + t < vis) ? __uint_as_float(sv[t]) * p.scale_log2 : -INFINITY;
@@ -309,9 +315,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       l_sum += acc;
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s_free[gp]);
       if (t0 + kT > L) {
         // value rows past the sequence may hold anything: zero them for PV
         const int tid = 32 * qd + lane;
