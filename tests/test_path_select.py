@@ -15,13 +15,13 @@ B200 = (148, 6559.0, 1656.2)   # SMs, copy GB/s, dense bf16 TFLOP/s (measured on
 # d = v = 128, B32, L 32K), measured on one B200 with `bench.py --sweep
 # crossover` (absorb ms, GQA ms).  A performance record, not an oracle value.
 MEASURED_B200 = {
-    (1, 1): (0.548, 0.190), (1, 2): (1.048, 0.356), (1, 4): (1.965, 0.674),
-    (2, 1): (0.549, 0.331), (2, 2): (1.048, 0.352), (2, 4): (1.965, 0.670),
-    (4, 1): (0.547, 0.478), (4, 2): (1.050, 0.630), (4, 4): (1.969, 0.667),
-    (8, 1): (0.549, 0.783), (8, 2): (1.050, 0.847), (8, 4): (1.972, 1.160),
-    (16, 1): (0.549, 1.493), (16, 2): (1.052, 1.508), (16, 4): (1.972, 1.597),
-    (32, 1): (0.553, 3.188), (32, 2): (1.054, 2.980), (32, 4): (1.984, 2.994),
-    (128, 1): (0.550, 12.688), (128, 2): (1.053, 12.515), (128, 4): (1.969, 12.587),
+    (1, 1): (0.525, 0.179), (1, 2): (1.005, 0.337), (1, 4): (1.880, 0.632),
+    (2, 1): (0.526, 0.312), (2, 2): (1.005, 0.331), (2, 4): (1.883, 0.631),
+    (4, 1): (0.524, 0.483), (4, 2): (1.005, 0.593), (4, 4): (1.882, 0.632),
+    (8, 1): (0.535, 0.779), (8, 2): (1.010, 0.846), (8, 4): (1.906, 1.110),
+    (16, 1): (0.545, 1.476), (16, 2): (1.006, 1.491), (16, 4): (1.883, 1.593),
+    (32, 1): (0.531, 3.183), (32, 2): (1.007, 2.936), (32, 4): (1.893, 2.950),
+    (128, 1): (0.526, 12.795), (128, 2): (1.008, 12.360), (128, 4): (1.884, 12.420),
 }
 
 
