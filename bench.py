@@ -296,6 +296,14 @@ def run_ours(args):
     def append_latent():
         gqla.gqla_append_tokens(dims, lay, new_rows, inp.latent, dev_status=status)
 
+    def append():
+        # the new rows into the latent pool, then their expansion into the per-group pools
+        gqla.gqla_append_tokens(dims, lay, new_rows, inp.latent, inp.W_uk, inp.W_uv, kp, vp, dev_status=status)
+
+    def expand_new():
+        # the new rows' expansion alone (no latent pool argument)
+        gqla.gqla_append_tokens(dims, lay, new_rows, None, inp.W_uk, inp.W_uv, kp, vp, dev_status=status)
+
     def expand_tail():
         gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, d.s_q, status)
 
@@ -307,27 +315,29 @@ def run_ours(args):
         gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out_g, lse_g, gqa_splits[0], ws_g, status)
 
     def step():
-        append_latent()
-        expand_tail()
+        append()
         absorb()
         gqa()
 
-    # The two paths of a step share no data once the new rows are in the
-    # latent pool: the absorb path runs on a second stream, forked from and
-    # joined back into the main one, so its CTAs and the GQA path's share the
-    # machine.
+    # The two paths of a step share no data once the new tokens are in the
+    # pools: the absorb path runs on a second stream, forked from and joined
+    # back into the main one, so its CTAs and the GQA path's share the machine.
     side = torch.cuda.Stream(dev)
 
-    def step_overlapped():
+    def step_overlapped(after_absorb=None, after_gqa=None):
         main = torch.cuda.current_stream(dev)   # the capture stream while a graph is recorded
-        append_latent()
+        append_latent()                         # what the absorb path needs ...
         fork = torch.cuda.Event()
         fork.record(main)
         side.wait_event(fork)
         with torch.cuda.stream(side):
             absorb()
-        expand_tail()
+            if after_absorb:
+                after_absorb()                  # e.g. its output's copy to the host, on the same stream
+        expand_new()                            # ... and what the GQA path needs, beside the absorb call
         gqa()
+        if after_gqa:
+            after_gqa()
         join = torch.cuda.Event()
         join.record(side)
         main.wait_event(join)
@@ -396,6 +406,7 @@ def run_ours(args):
     ms_gqa = timed(gqa, reps) / reps
     ms_tail = timed(expand_tail, reps) / reps
     ms_append = timed(append_latent, reps) / reps
+    ms_append_expand = timed(append, reps) / reps
     ms_expand_full = timed(lambda: gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0,
                                                           status), 3) / 3
     # the GQA call over the same cache with the RoPE key stored once per token
@@ -421,6 +432,13 @@ def run_ours(args):
         out_host[0].copy_(out_a, non_blocking=True)
         out_host[1].copy_(out_g, non_blocking=True)
 
+    def e2e_body_overlapped():
+        # each path's output goes to the host as soon as that path is done
+        inp.q.copy_(q_host, non_blocking=True)
+        new_rows.copy_(new_rows_host, non_blocking=True)
+        step_overlapped(after_absorb=lambda: out_host[0].copy_(out_a, non_blocking=True),
+                        after_gqa=lambda: out_host[1].copy_(out_g, non_blocking=True))
+
     absorb_splits[0], gqa_splits[0] = step_splits
     # the copies and the step's calls recorded once as a CUDA graph (the copies
     # read and write the pinned host buffers on every replay), then one replay
@@ -430,7 +448,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(e2e_graph):
-            e2e_body(step_overlapped)
+            e2e_body_overlapped()
 
     def e2e_step():
         if e2e_graph is not None:
@@ -490,8 +508,8 @@ def run_ours(args):
         "config": {"workload": "%s B%d L%d s_q%d" % (wl.name, B, wl.seq_len, d.s_q), "batch": B,
                    "seq_len": wl.seq_len, "s_q": d.s_q, "n_h": d.n_h, "G": d.G, "d_nope": d.d_nope,
                    "d_rope": d.d_rope, "d_v": d.d_v, "r": d.r,
-                   "step": ("append s_q new tokens to the latent cache + expand them + absorb decode + "
-                            "GQA decode"),
+                   "step": ("append the s_q new tokens (latent rows + their per-group expansion) + absorb "
+                            "decode + GQA decode"),
                    "launch": ("cuda_graph replay of the step; absorb path on a second stream, overlapped with "
                               "the tail expansion + GQA path") if graph is not None else "eager, sequential",
                    "eager_ms_per_step": eager_ms,
@@ -513,6 +531,7 @@ def run_ours(args):
                   "gqa_shared_rope": path_entry(ms_gqa_s, alg["gqa_shared_bytes"], alg["gqa_flops"]),
                   "expand_tail": {"ms": ms_tail},
                   "append_latent": {"ms": ms_append},
+                  "append_and_expand": {"ms": ms_append_expand},
                   "expand_full_cache": {"ms": ms_expand_full, "tflops": exp_flops / (ms_expand_full * 1e-3) / 1e12,
                                         "hbm_gbs": exp_bytes / (ms_expand_full * 1e-3) / 1e9,
                                         "tc_frac": exp_flops / (ms_expand_full * 1e-3) / (tf_burst * 1e12)}},

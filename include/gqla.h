@@ -152,9 +152,15 @@ gqla_status gqla_expand_cache(const gqla_dims* dims, const gqla_kv_layout* layou
  * count the new tokens), and, when k_pool and v_pool are given, those tokens
  * are expanded into the per-group pools as gqla_expand_cache does.
  *   new_rows  device [B, s_q, r + d_rope]
- *   latent    device pool (written at the new positions only)
+ *   latent    device pool (written at the new positions only), or NULL for
+ *             a GQA-only cache: then only the expansion happens (bf16 dims
+ *             of the tensor-core kernels only; else GQLA_ERR_UNSUPPORTED)
  *   W_uk, W_uv, k_pool, v_pool  as for gqla_expand_cache; k_pool/v_pool may
  *             both be NULL (absorb-only cache), then W_uk/W_uv are unused.
+ *             latent and k_pool may not both be NULL.
+ * With the tensor-core kernels the expansion reads the dense new_rows, many
+ * sequences' tokens to an MMA tile; each token's K/V rows are the same
+ * numbers gqla_expand_cache produces for it.
  * A sequence shorter than s_q, longer than its slots or with a page outside
  * the pool is skipped and flagged in *dev_status. */
 gqla_status gqla_append_tokens(const gqla_dims* dims, const gqla_kv_layout* layout, const void* new_rows,

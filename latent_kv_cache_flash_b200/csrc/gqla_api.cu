@@ -277,16 +277,21 @@ gqla_status gqla_append_tokens(const gqla_dims* dims, const gqla_kv_layout* layo
   Problem p;
   gqla_status s = make_problem(dims, layout, 1, GQLA_PATH_GQA, &p);
   if (s != GQLA_OK) return s;
-  if (!new_rows || !latent) return GQLA_ERR_INVALID_ARG;
+  if (!new_rows) return GQLA_ERR_INVALID_ARG;
   const bool expand = k_pool || v_pool;
+  if (!latent && !expand) return GQLA_ERR_INVALID_ARG;
   if (expand && (!k_pool || !v_pool || !W_uk || !W_uv)) return GQLA_ERR_INVALID_ARG;
-  if (!aligned16(new_rows) || !aligned16(latent)) return GQLA_ERR_ALIGNMENT;
+  if (!aligned16(new_rows) || (latent && !aligned16(latent))) return GQLA_ERR_ALIGNMENT;
   if (expand && (!aligned16(W_uk) || !aligned16(W_uv) || !aligned16(k_pool) || !aligned16(v_pool)))
     return GQLA_ERR_ALIGNMENT;
+  // without a latent pool the expansion must read the dense new rows
+  if (!latent && !tc_expand_supports(p)) return GQLA_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = append_rows(p, new_rows, latent, dev_status, st);
+  cudaError_t e = latent ? append_rows(p, new_rows, latent, dev_status, st) : cudaSuccess;
   if (e == cudaSuccess && expand) {
-    if (tc_expand_supports(p)) e = tc_expand(p, latent, W_uk, W_uv, k_pool, v_pool, p.d.s_q, dev_status, st);
+    // the new rows are dense: the tensor-core form packs many sequences' new
+    // tokens into each 128-row tile
+    if (tc_expand_supports(p)) e = tc_expand_dense(p, new_rows, k_pool, v_pool, W_uk, W_uv, dev_status, st);
     else e = simt_expand(p, latent, W_uk, W_uv, k_pool, v_pool, p.d.s_q, dev_status, st);
   }
   return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;

@@ -45,6 +45,10 @@ cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const f
 
 // Cache expansion GEMM on tcgen05 (tc_expand.cu).
 bool tc_expand_supports(const Problem& p);
+// Expansion of a dense matrix of the B * s_q new token rows (row b * s_q + i
+// is token seq_lens[b] - s_q + i), written to those tokens' pool rows.
+cudaError_t tc_expand_dense(const Problem& p, const void* rows, void* k_pool, void* v_pool, const void* W_uk,
+                            const void* W_uv, int32_t* st, cudaStream_t s);
 cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, const void* W_uv, void* k_pool,
                       void* v_pool, int tail, int32_t* st, cudaStream_t s);
 

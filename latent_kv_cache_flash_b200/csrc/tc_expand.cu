@@ -16,6 +16,13 @@
 //    round to bf16 and write the K and V rows, and copy the shared RoPE key.
 // Tiles start on a 64-token boundary; rows outside [first token, L) of the
 // sequence are computed but not written.
+//
+// A second form takes a dense matrix of token rows instead of the pool (the
+// s_q new rows of every sequence, B * s_q of them, at decode time): its
+// tiles are 128 consecutive rows of that matrix, so the new tokens of many
+// sequences share one tile, and each output row goes to its token's pool
+// row.  The MMA shapes and the order over K are the same in both forms, so a
+// token's expansion is the same numbers whichever form produced it.
 #include "ptx.cuh"
 #include "tc.h"
 
@@ -47,14 +54,36 @@ struct ExpandParams {
   int G;
   int tail;          // > 0: only the newest `tail` tokens of each sequence
   int tps;           // tiles per sequence
-  long long n_items; // batch * tps * G
+  long long n_items; // batch * tps * G  (dense form: ceil(dense_rows / 128) * G)
+  const bf16* dense; // dense form: [dense_rows, 576] new rows, row b * s_q + i = token L_b - s_q + i
+  int dense_rows;    // 0: pool form
+  int s_q;
   int32_t* st;
 };
 
+// Dense form: pool row of dense row dr (= b * s_q + i), or -1 when the
+// sequence is invalid or the page is outside the pool (flagged).
+__device__ __forceinline__ long long dense_row_target(const ExpandParams& p, int dr) {
+  const KvLayout& ly = p.ly;
+  const int b = dr / p.s_q, i = dr % p.s_q;
+  const int L = ly.seq_lens[b];
+  const bool bad = L < p.s_q || L > ly.max_seq_len ||
+                   (ly.page_size == 0 ? L > ly.capacity : (L + ly.page_size - 1) / ly.page_size > ly.mbps);
+  if (bad) return -1;
+  return token_row(ly, b, L - p.s_q + i, p.st);
+}
+
 // Tile j of sequence b: first token t0 (64-aligned) and the token range
-// [t_lo, t_hi) that is written.  Returns false when the item is empty.
+// [t_lo, t_hi) that is written.  Returns false when the item is empty.  In
+// the dense form "sequence" 0 has tiles of 128 dense rows: t0 is the first.
 __device__ __forceinline__ bool item_tile(const ExpandParams& p, int b, int j, int* t0, int* t_lo, int* t_hi,
                                           bool report = false) {
+  if (p.dense_rows > 0) {
+    *t0 = j * kTM;
+    *t_lo = 0;
+    *t_hi = p.dense_rows;
+    return *t0 < p.dense_rows;
+  }
   const KvLayout& ly = p.ly;
   const int L = ly.seq_lens[b];
   const bool bad = L < 1 || L > ly.max_seq_len ||
@@ -126,7 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = (int)(bt / p.tps), j = (int)(bt % p.tps);
         int t0, tlo, thi;
         if (!item_tile(p, b, j, &t0, &tlo, &thi, g == 0)) continue;
-        const int row0 = half_row(p.ly, b, t0, thi), row1 = half_row(p.ly, b, t0 + 64, thi);
+        // dense form: rows of the dense matrix (a box past its end reads zeros)
+        const int row0 = p.dense_rows > 0 ? t0 : half_row(p.ly, b, t0, thi);
+        const int row1 = p.dense_rows > 0 ? t0 + 64 : half_row(p.ly, b, t0 + 64, thi);
         for (int kc = 0; kc < kR / kKC; ++kc, ++it) {
           const int s = (int)(it % kStages);
           const long long k = it / kStages;
@@ -212,9 +243,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = ptx::mbar_wait(&acc_full[ab], (uint32_t)((li >> 1) & 1));
       ok = __all_sync(0xffffffffu, ok);
       const int t = t0 + r;
-      const bool write = ok && t >= tlo && t < thi;
+      bool write = ok && t >= tlo && t < thi;
       long long row = 0;
-      if (write) row = half_row(p.ly, b, t0 + (r & ~63), thi) + (r & 63);
+      if (write) {
+        if (p.dense_rows > 0) {
+          row = dense_row_target(p, t);
+          write = row >= 0;
+        } else {
+          row = half_row(p.ly, b, t0 + (r & ~63), thi) + (r & 63);
+        }
+      }
       if (ok) {
         ptx::tc_fence_after();
 #pragma unroll 1
@@ -237,7 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (write && (p.kr.rope_gs != 0 || g == 0)) {   // a shared RoPE key is written by group 0
-          const uint4* src = reinterpret_cast<const uint4*>(p.latent + row * kE + kR);
+          const uint4* src = reinterpret_cast<const uint4*>(p.dense_rows > 0 ? p.dense + (long long)t * kE + kR
+                                                                             : p.latent + row * kE + kR);
           uint4* dst = reinterpret_cast<uint4*>(p.kp + row * p.kr.pitch + p.kr.rope_at(g));
 #pragma unroll
           for (int e = 0; e < kDr / 8; ++e) dst[e] = src[e];
@@ -291,11 +330,46 @@ cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, co
   prm.tail = tail > 0 ? span : 0;
   prm.tps = (span + 63 + kTM - 1) / kTM;
   prm.n_items = (long long)p.ly.batch * prm.tps * d.G;
+  prm.dense = nullptr;
+  prm.dense_rows = 0;
+  prm.s_q = d.s_q;
   prm.st = st;
   cudaError_t e = ensure_smem_limit((const void*)expand_tc_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long grid = prm.n_items < num_sms() ? prm.n_items : num_sms();
   if (grid < 1) return cudaSuccess;
+  expand_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(lat_map, uk_map, uv_map, prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t tc_expand_dense(const Problem& p, const void* rows, void* k_pool, void* v_pool, const void* W_uk,
+                            const void* W_uv, int32_t* st, cudaStream_t s) {
+  const auto& d = p.d;
+  const long long n = (long long)p.ly.batch * d.s_q;
+  if (n > (1LL << 30)) return cudaErrorInvalidValue;
+  CUtensorMap lat_map, uk_map, uv_map;
+  if (!tmap_bf16_sw128(&lat_map, rows, kE, n, kE, 64) ||
+      !tmap_bf16_sw128(&uk_map, W_uk, kDn, (long long)d.G * kR, kDn, kKC) ||
+      !tmap_bf16_sw128(&uv_map, W_uv, kDv, (long long)d.G * kR, kDv, kKC))
+    return cudaErrorInvalidValue;
+  ExpandParams prm;
+  prm.ly = p.ly;
+  prm.kp = (bf16*)k_pool;
+  prm.kr = p.kr;
+  prm.vp = (bf16*)v_pool;
+  prm.latent = nullptr;
+  prm.G = d.G;
+  prm.tail = 0;
+  prm.tps = (int)((n + kTM - 1) / kTM);
+  prm.n_items = (long long)prm.tps * d.G;
+  prm.dense = (const bf16*)rows;
+  prm.dense_rows = (int)n;
+  prm.s_q = d.s_q;
+  prm.st = st;
+  cudaError_t e = ensure_smem_limit((const void*)expand_tc_kernel, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const long long grid = prm.n_items < num_sms() ? prm.n_items : num_sms();
   expand_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(lat_map, uk_map, uv_map, prm);
   count_launch();
   return cudaGetLastError();

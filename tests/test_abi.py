@@ -111,6 +111,13 @@ def test_validation_before_launch(G):
                                 None) == G.GQLA_ERR_INVALID_ARG
     assert L.gqla_append_tokens(ctypes.byref(d), ctypes.byref(lay), p, a, null, null, null, null, None,
                                 None) == G.GQLA_ERR_ALIGNMENT
+    # neither a latent pool nor expanded pools: nothing to write
+    assert L.gqla_append_tokens(ctypes.byref(d), ctypes.byref(lay), a, null, a, a, null, null, None,
+                                None) == G.GQLA_ERR_INVALID_ARG
+    # expansion without a latent pool needs the tensor-core kernels (bf16 dims)
+    f32 = _dims(G, dtype=G.GQLA_F32)
+    assert L.gqla_append_tokens(ctypes.byref(f32), ctypes.byref(lay), a, null, a, a, a, a, None,
+                                None) == G.GQLA_ERR_UNSUPPORTED
 
 
 def test_split_plan_and_workspace(G):

@@ -109,6 +109,27 @@ def test_append_latent_only_leaves_pools_alone():
     assert torch.equal(inp.latent, ref_latent)
 
 
+def test_append_expansion_only_without_latent_pool():
+    """latent = NULL: the GQA-only cache gets the new tokens' K/V from the
+    dense rows alone, bit for bit as the full expansion gives them."""
+    d = synth.Dims(**LLAMA, s_q=3)
+    inp = _inputs(d, [500, 3, 64, 1000], 64, seed=53)
+    kp_ref, vp_ref = H.run_expand(inp)
+    new_rows = _new_rows(inp)
+    before = inp.latent.clone()
+    kp, vp = kp_ref.clone(), vp_ref.clone()
+    _poison_new_slots(kp, inp)
+    _poison_new_slots(vp, inp)
+    from latent_kv_cache_flash_b200 import gqla
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gqla.gqla_append_tokens(gqla.make_dims(inp.dims), H.layout_of(inp), new_rows, None, inp.W_uk, inp.W_uv, kp, vp,
+                            dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(kp, kp_ref) and torch.equal(vp, vp_ref)
+    assert torch.equal(inp.latent, before)
+
+
 def test_append_f32_contiguous():
     d = synth.Dims(n_h=8, G=2, d_nope=32, d_rope=16, d_v=32, r=64, s_q=3, dtype="f32")
     inp = _inputs(d, [5, 3, 70], 0, seed=51)
