@@ -149,7 +149,7 @@ size_t ws_layout(const Problem& p, gqla_path path, bool tc, Workspace* ws, char*
   size_t off = 0;
   const int S = p.plan.num_splits;
   const int D = path == GQLA_PATH_ABSORB ? p.d.r : p.d.d_v;
-  Workspace w{nullptr, nullptr, nullptr, nullptr};
+  Workspace w{nullptr, nullptr, nullptr, nullptr, nullptr};
   auto take = [&](size_t bytes) {
     void* ptr = base ? base + off : nullptr;
     off = align256(off + bytes);
@@ -163,6 +163,10 @@ size_t ws_layout(const Problem& p, gqla_path path, bool tc, Workspace* ws, char*
   if (S > 1 || (tc && path == GQLA_PATH_ABSORB)) {
     w.o_part = (float*)take((size_t)S * p.rows * D * 4);
     w.lse_part = (float*)take((size_t)S * p.rows * 4);
+  }
+  if (S > 1 && path == GQLA_PATH_GQA) {
+    const long long blocks = (long long)p.ly.batch * p.d.G * ((p.m * p.d.s_q + 15) / 16);
+    w.counters = (int*)take((size_t)blocks * 4);
   }
   if (ws) *ws = w;
   return off;
@@ -205,6 +209,20 @@ int num_sms() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+cudaError_t gqa_decode_call(const Problem& p, bool tc, const void* q, const void* k_pool, const void* v_pool,
+                            void* out, float* lse, const Workspace& w, int32_t* st, cudaStream_t s) {
+  const int S = p.plan.num_splits;
+  cudaError_t e;
+  bool merged = false;
+  if (tc) e = tc_gqa_decode(p, q, k_pool, v_pool, S > 1 ? nullptr : out, S > 1 ? w.o_part : nullptr,
+                            S > 1 ? w.lse_part : lse, st, s, w.counters, out, lse, &merged);
+  else e = simt_decode(p, GQLA_PATH_GQA, q, nullptr, k_pool, v_pool, S > 1 ? nullptr : out,
+                       S > 1 ? w.o_part : nullptr, S > 1 ? w.lse_part : lse, st, s);
+  if (e == cudaSuccess && S > 1 && !merged)
+    e = combine(S, p.rows, p.d.d_v, w.o_part, w.lse_part, out, p.d.dtype, lse, s);
+  return e;
 }
 
 }  // namespace gqla
@@ -319,16 +337,10 @@ gqla_status gqla_decode_gqa(const gqla_dims* dims, const gqla_kv_layout* layout,
   Workspace w;
   size_t need = ws_layout(p, GQLA_PATH_GQA, false, &w, (char*)workspace);
   if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u))) return GQLA_ERR_WORKSPACE;
-  cudaStream_t st = (cudaStream_t)stream;
-  const int S = p.plan.num_splits;
-  cudaError_t e;
-  if (tc) e = tc_gqa_decode(p, q, k_pool, v_pool, S > 1 ? nullptr : out, S > 1 ? w.o_part : nullptr,
-                            S > 1 ? w.lse_part : lse, dev_status, st);
-  else e = simt_decode(p, GQLA_PATH_GQA, q, nullptr, k_pool, v_pool, S > 1 ? nullptr : out,
-                       S > 1 ? w.o_part : nullptr, S > 1 ? w.lse_part : lse, dev_status, st);
-  if (e == cudaSuccess && S > 1) e = combine(S, p.rows, p.d.d_v, w.o_part, w.lse_part, out, p.d.dtype, lse, st);
+  cudaError_t e = gqa_decode_call(p, tc, q, k_pool, v_pool, out, lse, w, dev_status, (cudaStream_t)stream);
   return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;
 }
+
 
 gqla_status gqla_decode_absorb(const gqla_dims* dims, const gqla_kv_layout* layout, const void* q,
                                const void* latent, const void* W_uk, const void* W_uv, void* out, float* lse,

@@ -71,15 +71,9 @@ extern "C" gqla_status gqla_decode_gqa_noalloc(const gqla_dims* dims, const gqla
   }
   Workspace w;
   ws_layout(p, GQLA_PATH_GQA, false, &w, (char*)scratch);
-  cudaStream_t st = (cudaStream_t)stream;
-  const int S = p.plan.num_splits;
   // Every split writes its whole partial (an empty split writes zeros and
-  // lse = -inf), so nothing left in the scratch by an earlier call is read.
-  cudaError_t e;
-  if (tc) e = tc_gqa_decode(p, q, k_pool, v_pool, S > 1 ? nullptr : out, S > 1 ? w.o_part : nullptr,
-                            S > 1 ? w.lse_part : lse, dev_status, st);
-  else e = simt_decode(p, GQLA_PATH_GQA, q, nullptr, k_pool, v_pool, S > 1 ? nullptr : out,
-                       S > 1 ? w.o_part : nullptr, S > 1 ? w.lse_part : lse, dev_status, st);
-  if (e == cudaSuccess && S > 1) e = combine(S, p.rows, p.d.d_v, w.o_part, w.lse_part, out, p.d.dtype, lse, st);
+  // lse = -inf) and the split counters are zeroed before the launch, so
+  // nothing left in the scratch by an earlier call is read.
+  cudaError_t e = gqa_decode_call(p, tc, q, k_pool, v_pool, out, lse, w, dev_status, (cudaStream_t)stream);
   return e == cudaSuccess ? GQLA_OK : GQLA_ERR_CUDA;
 }

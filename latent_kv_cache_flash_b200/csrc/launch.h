@@ -30,7 +30,13 @@ struct Workspace {
   float* o_part;   // [S, rows, D] when S > 1
   float* lse_part; // [S, rows] when S > 1
   float* o_lat;    // absorb: combined latent outputs [rows, r]
+  int* counters;   // GQA with S > 1: split counts per (sequence, group, row block)
 };
+
+// The GQA call from its workspace: decode (and the split merge, in the
+// kernel or as a combine pass).  Shared by the workspace and no-alloc entries.
+cudaError_t gqa_decode_call(const Problem& p, bool tc, const void* q, const void* k_pool, const void* v_pool,
+                            void* out, float* lse, const Workspace& w, int32_t* st, cudaStream_t s);
 
 // Validates dims/layout and builds the problem with its split plan.
 gqla_status make_problem(const gqla_dims* dims, const gqla_kv_layout* layout, int num_splits, gqla_path path,

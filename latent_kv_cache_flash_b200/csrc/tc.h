@@ -18,8 +18,12 @@ bool gqa_pool_maps(const Problem& p, const void* k_pool, const void* v_pool, CUt
 // GQA decode over the expanded cache: mma.sync bf16 tiles, cp.async.bulk
 // staged K/V pages, online softmax per 16-row block.
 bool tc_gqa_supports(const Problem& p);
+// With split partials (o_part) and a counter array of B * G * ceil(m s_q / 16)
+// ints, the mma.sync kernel merges the splits itself into out_final /
+// lse_final and sets *merged; otherwise the caller runs the combine.
 cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
-                          float* o_part, float* lse_dst, int32_t* st, cudaStream_t s);
+                          float* o_part, float* lse_dst, int32_t* st, cudaStream_t s, int* counters = nullptr,
+                          void* out_final = nullptr, float* lse_final = nullptr, bool* merged = nullptr);
 
 // GQA decode for m * s_q >= 64 rows per group: tcgen05/TMEM (tc_gqa_wide.cu);
 // tc_gqa_decode hands such problems to it.

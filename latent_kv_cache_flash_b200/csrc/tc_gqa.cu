@@ -17,7 +17,11 @@
 //    mma.sync m16n8k16 bf16 (fp32 accumulate) from ldmatrix'd fragments, and
 //    keep an online softmax (running max in the log2 domain) per row;
 //  * the warps' partial states are merged through shared memory at the end;
-//    the result goes to `out` (one split) or to fp32 split partials.
+//    the result goes to `out` (one split) or to fp32 split partials.  With
+//    split partials, the last CTA of a (sequence, group, row block) to finish
+//    (an atomic count per block) merges all splits' partials by their
+//    log-sum-exp and writes the final output, so no separate combine pass
+//    re-reads them.
 #include <math.h>
 
 #include "ptx.cuh"
@@ -54,6 +58,11 @@ struct GqaParams {
   float scale_log2;
   long long rows;  // B * s_q * n_h
   int32_t* st;
+  // split merge in the kernel (o_part != nullptr): counters zeroed before
+  // the launch, one per (sequence, group, CTA row block); final outputs
+  int* counters;
+  __nv_bfloat16* out_final;
+  float* lse_final;
 };
 
 static_assert(kConsumerWarps * 16 * kOStride * 4 + 2 * kConsumerWarps * 16 * 4 <= kStages * kStageBytes,
@@ -320,6 +329,48 @@ __global__ void __launch_bounds__(kThreads, 2)
       p.lse[p.o_part ? (long long)split * p.rows + gr : gr] = lse;
     }
   }
+  if (p.o_part && p.counters) {
+    // ------------------------------------ merge the splits (last CTA only)
+    __shared__ int last_cta;
+    __threadfence();                              // this CTA's partials are visible before the count
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+    const int S = p.plan.num_splits;
+    int* counter = p.counters + ((long long)blockIdx.y * gridDim.z + blockIdx.z);
+    if (tid == 0) last_cta = atomicAdd(counter, 1) == S - 1;
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+    if (last_cta) {
+      __threadfence();
+      for (int idx = tid; idx < p.rbc * 16 * (kDv / 4); idx += kConsumerWarps * 32) {
+        const int rl = idx / (kDv / 4), d4 = (idx % (kDv / 4)) * 4;
+        const int r = rb0 * 16 + rl;
+        if (r >= p.rows_unit) continue;
+        const int i = r / p.m, h = g * p.m + r % p.m;
+        const long long gr = ((long long)b * p.s_q + i) * p.n_h + h;
+        float mx = -INFINITY;
+        for (int sp = 0; sp < S; ++sp) mx = fmaxf(mx, __ldcg(p.lse + (long long)sp * p.rows + gr));
+        float z = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (mx != -INFINITY) {
+          for (int sp = 0; sp < S; ++sp) {
+            const float ls = __ldcg(p.lse + (long long)sp * p.rows + gr);
+            if (ls == -INFINITY) continue;
+            const float w = expf(ls - mx);
+            z += w;
+            const float4 o = __ldcg(reinterpret_cast<const float4*>(p.o_part + ((long long)sp * p.rows + gr) * kDv + d4));
+            acc.x = fmaf(w, o.x, acc.x);
+            acc.y = fmaf(w, o.y, acc.y);
+            acc.z = fmaf(w, o.z, acc.z);
+            acc.w = fmaf(w, o.w, acc.w);
+          }
+        }
+        const float inv = z > 0.f ? 1.f / z : 0.f;
+        *reinterpret_cast<uint2*>(p.out_final + gr * kDv + d4) =
+            make_uint2(ptx::pack_bf16(acc.x * inv, acc.y * inv), ptx::pack_bf16(acc.z * inv, acc.w * inv));
+        if (d4 == 0 && p.lse_final) p.lse_final[gr] = mx == -INFINITY ? -INFINITY : mx + logf(z);
+      }
+      if (tid == 0) *counter = 0;                 // back to zero for the next call
+    }
+  }
 }
 
 }  // namespace
@@ -334,7 +385,9 @@ bool tc_gqa_supports(const Problem& p) {
 }
 
 cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
-                          float* o_part, float* lse_dst, int32_t* st, cudaStream_t s) {
+                          float* o_part, float* lse_dst, int32_t* st, cudaStream_t s, int* counters,
+                          void* out_final, float* lse_final, bool* merged) {
+  if (merged) *merged = false;
   if (tc_gqa_wide_supports(p)) return tc_gqa_wide_decode(p, q, k_pool, v_pool, out, o_part, lse_dst, st, s);
   const auto& d = p.d;
   CUtensorMap kmap, vmap;
@@ -358,10 +411,19 @@ cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, c
   prm.st = st;
   prm.kr = p.kr;
   dim3 grid(p.plan.num_splits, p.ly.batch * d.G, (rb + prm.rbc - 1) / prm.rbc);
+  const bool merge = o_part && counters && out_final;
+  prm.counters = merge ? counters : nullptr;
+  prm.out_final = (__nv_bfloat16*)out_final;
+  prm.lse_final = lse_final;
+  if (merge) {
+    cudaError_t e0 = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)grid.y * grid.z, s);
+    if (e0 != cudaSuccess) return e0;
+  }
   cudaError_t e = ensure_smem_limit((const void*)gqa_decode_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   gqa_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, prm);
   count_launch();
+  if (merge && merged) *merged = true;
   return cudaGetLastError();
 }
 
