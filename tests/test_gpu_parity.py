@@ -193,7 +193,8 @@ def test_edge_lengths(path):
 
 
 @pytest.mark.parametrize("path", ["absorb", "gqa"])
-def test_device_status_flags(path):
+@pytest.mark.parametrize("splits", [0, 3])
+def test_device_status_flags(path, splits):
     from latent_kv_cache_flash_b200 import gqla
     d = synth.Dims(**LLAMA, s_q=2)
     inp = _wl(d, 3, [100, 200, 300], page=64, seed=1)
@@ -201,7 +202,7 @@ def test_device_status_flags(path):
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
     inp.seq_lens[0] = 1                       # shorter than s_q
     inp.block_table[2, 1] = inp.num_pages + 5  # page id outside the pool
-    out, lse = H.run_decode(inp, path, pools=pools, dev_status=st)
+    out, lse = H.run_decode(inp, path, pools=pools, dev_status=st, num_splits=splits)
     torch.cuda.synchronize()
     flags = int(st.item())
     assert flags & gqla.DEV_SHORT_SEQ and flags & gqla.DEV_BAD_PAGE
@@ -212,7 +213,7 @@ def test_device_status_flags(path):
     H.check_units(inp, out, lse, [(1, g) for g in range(d.G)], "healthy row " + path)
     st.zero_()
     inp.seq_lens[1] = 400                     # above the host bound max_seq_len=300
-    H.run_decode(inp, path, pools=pools, dev_status=st, max_seq_len=300)
+    H.run_decode(inp, path, pools=pools, dev_status=st, max_seq_len=300, num_splits=splits)
     torch.cuda.synchronize()
     assert int(st.item()) & gqla.DEV_OVERFLOW
 
