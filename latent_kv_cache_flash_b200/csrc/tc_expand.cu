@@ -21,8 +21,11 @@
 // s_q new rows of every sequence, B * s_q of them, at decode time): its
 // tiles are 128 consecutive rows of that matrix, so the new tokens of many
 // sequences share one tile, and each output row goes to its token's pool
-// row.  The MMA shapes and the order over K are the same in both forms, so a
-// token's expansion is the same numbers whichever form produced it.
+// row.  A dense item may also cover only the K or only the V half of the
+// outputs (N = 128), so that a small batch of new tokens spreads over twice
+// as many CTAs, each loading half the weights.  Every output element is
+// still the same K-ordered sum of bf16 products, so a token's expansion is
+// the same numbers whichever form produced it.
 #include "ptx.cuh"
 #include "tc.h"
 
@@ -57,6 +60,7 @@ struct ExpandParams {
   long long n_items; // batch * tps * G  (dense form: ceil(dense_rows / 128) * G)
   const bf16* dense; // dense form: [dense_rows, 576] new rows, row b * s_q + i = token L_b - s_q + i
   int dense_rows;    // 0: pool form
+  int halves;        // 2: an item covers the K or the V outputs only (item % 2), else both
   int s_q;
   int32_t* st;
 };
@@ -150,8 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long it = 0;
       bool ok = true;
       for (long long item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int g = (int)(item % G);
-        const long long bt = item / G;
+        const int hf = p.halves == 2 ? (int)(item & 1) : -1;
+        const long long it2 = p.halves == 2 ? item >> 1 : item;
+        const int g = (int)(it2 % G);
+        const long long bt = it2 / G;
         const int b = (int)(bt / p.tps), j = (int)(bt % p.tps);
         int t0, tlo, thi;
         if (!item_tile(p, b, j, &t0, &tlo, &thi, g == 0)) continue;
@@ -167,15 +173,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* st = smem + s * kStageBytes;
-          ptx::mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
+          ptx::mbar_arrive_expect_tx(&full_bar[s], hf < 0 ? kStageBytes : kABytes + 2 * kBBox);
           ptx::tma_load_2d(st, &lat_map, &full_bar[s], kKC * kc, row0);
           ptx::tma_load_2d(st + kABytes / 2, &lat_map, &full_bar[s], kKC * kc, row1);
           uint8_t* bs = st + kABytes;
           const int wrow = g * kR + kKC * kc;
-          ptx::tma_load_2d(bs + 0 * kBBox, &uk_map, &full_bar[s], 0, wrow);
-          ptx::tma_load_2d(bs + 1 * kBBox, &uk_map, &full_bar[s], 64, wrow);
-          ptx::tma_load_2d(bs + 2 * kBBox, &uv_map, &full_bar[s], 0, wrow);
-          ptx::tma_load_2d(bs + 3 * kBBox, &uv_map, &full_bar[s], 64, wrow);
+          if (hf != 1) {
+            ptx::tma_load_2d(bs + 0 * kBBox, &uk_map, &full_bar[s], 0, wrow);
+            ptx::tma_load_2d(bs + 1 * kBBox, &uk_map, &full_bar[s], 64, wrow);
+          }
+          if (hf != 0) {
+            const int vb = hf < 0 ? 2 : 0;       // V boxes after the K boxes, or alone
+            ptx::tma_load_2d(bs + (vb + 0) * kBBox, &uv_map, &full_bar[s], 0, wrow);
+            ptx::tma_load_2d(bs + (vb + 1) * kBBox, &uv_map, &full_bar[s], 64, wrow);
+          }
         }
       }
       // no copy may still be landing when the CTA retires
@@ -185,16 +196,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_bf16(kTM, kN, false, true);
+      constexpr uint32_t idesc_full = ptx::idesc_bf16(kTM, kN, false, true);
+      constexpr uint32_t idesc_half = ptx::idesc_bf16(kTM, kN / 2, false, true);
       const uint32_t base = ptx::smem_u32(smem);
       long long it = 0, li = 0;
       bool ok = true;
       for (long long item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int g = (int)(item % G);
-        const long long bt = item / G;
+        const int hf = p.halves == 2 ? (int)(item & 1) : -1;
+        const long long it2 = p.halves == 2 ? item >> 1 : item;
+        const int g = (int)(it2 % G);
+        const long long bt = it2 / G;
         const int b = (int)(bt / p.tps), j = (int)(bt % p.tps);
         int t0, tlo, thi;
         (void)g;
+        const uint32_t idesc = hf < 0 ? idesc_full : idesc_half;
         if (!item_tile(p, b, j, &t0, &tlo, &thi)) continue;
         const int ab = (int)(li & 1);
         if (li >= 2 && !ptx::mbar_wait(&acc_empty[ab], (uint32_t)(((li >> 1) - 1) & 1))) {
@@ -234,8 +249,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long li = 0;
     bool ok = true;
     for (long long item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-      const int g = (int)(item % G);
-      const long long bt = item / G;
+      const int hf = p.halves == 2 ? (int)(item & 1) : -1;
+      const long long it2 = p.halves == 2 ? item >> 1 : item;
+      const int g = (int)(it2 % G);
+      const long long bt = it2 / G;
       const int b = (int)(bt / p.tps), j = (int)(bt % p.tps);
       int t0, tlo, thi;
       if (!item_tile(p, b, j, &t0, &tlo, &thi)) continue;
@@ -255,14 +272,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok) {
         ptx::tc_fence_after();
+        const int ncol = hf < 0 ? kN / 32 : kN / 64;   // 32-column groups in the accumulator
 #pragma unroll 1
-        for (int c = 0; c < kN / 32; ++c) {
+        for (int c = 0; c < ncol; ++c) {
           uint32_t v[32];
           ptx::tmem_ld32(tl + (uint32_t)(ab * kN + 32 * c), v);
           ptx::tmem_ld_wait();
           if (write) {
-            bf16* dst = c < kDn / 32 ? p.kp + row * p.kr.pitch + p.kr.nope_at(g) + 32 * c
-                                     : p.vp + (row * G + g) * kDv + 32 * (c - kDn / 32);
+            const int oc = hf == 1 ? c + kDn / 32 : c;   // column group of [K nope | V]
+            bf16* dst = oc < kDn / 32 ? p.kp + row * p.kr.pitch + p.kr.nope_at(g) + 32 * oc
+                                      : p.vp + (row * G + g) * kDv + 32 * (oc - kDn / 32);
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               uint4 w;
@@ -274,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (write && (p.kr.rope_gs != 0 || g == 0)) {   // a shared RoPE key is written by group 0
+        if (write && hf != 1 && (p.kr.rope_gs != 0 || g == 0)) {   // a shared RoPE key: by group 0
           const uint4* src = reinterpret_cast<const uint4*>(p.dense_rows > 0 ? p.dense + (long long)t * kE + kR
                                                                              : p.latent + row * kE + kR);
           uint4* dst = reinterpret_cast<uint4*>(p.kp + row * p.kr.pitch + p.kr.rope_at(g));
@@ -332,6 +351,7 @@ cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, co
   prm.n_items = (long long)p.ly.batch * prm.tps * d.G;
   prm.dense = nullptr;
   prm.dense_rows = 0;
+  prm.halves = 1;
   prm.s_q = d.s_q;
   prm.st = st;
   cudaError_t e = ensure_smem_limit((const void*)expand_tc_kernel, (int)kSmemBytes);
@@ -362,7 +382,8 @@ cudaError_t tc_expand_dense(const Problem& p, const void* rows, void* k_pool, vo
   prm.G = d.G;
   prm.tail = 0;
   prm.tps = (int)((n + kTM - 1) / kTM);
-  prm.n_items = (long long)prm.tps * d.G;
+  prm.halves = 2;
+  prm.n_items = (long long)prm.tps * d.G * prm.halves;
   prm.dense = (const bf16*)rows;
   prm.dense_rows = (int)n;
   prm.s_q = d.s_q;
