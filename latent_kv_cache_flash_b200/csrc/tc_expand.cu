@@ -12,8 +12,12 @@
 //    weight matrices) into a 4-stage mbarrier ring;
 //  * warp 1 issues 4 tcgen05.mma (M=128, N=256, K=16; A K-major, B MN-major)
 //    per chunk into one of two TMEM accumulators (2 x 256 columns);
-//  * warps 2-5 drain an accumulator (tcgen05.ld, one token row per thread),
-//    round to bf16 and write the K and V rows, and copy the shared RoPE key.
+//  * warps 2-5 drain an accumulator (tcgen05.ld, one token row per thread)
+//    and round to bf16.  A 64-token half tile whose rows are all written
+//    goes through a 128-byte-swizzled staging tile to TMA stores of 64 x 64
+//    boxes (each row from one thread would make every warp store touch 32
+//    rows G * 640 bytes apart); other rows are stored by their thread.  The
+//    shared RoPE key is copied by the threads.
 // Tiles start on a 64-token boundary; rows outside [first token, L) of the
 // sequence are computed but not written.
 //
@@ -39,12 +43,14 @@ constexpr int kR = 512, kDn = 128, kDv = 128, kDr = 64, kE = kR + kDr;
 constexpr int kTM = 128;                          // tokens per tile
 constexpr int kN = kDn + kDv;                     // 256 outputs per group
 constexpr int kKC = 64;                           // K per stage
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kABytes = kTM * 128;                // 16 KB
 constexpr int kBBox = kKC * 128;                  // 8 KB: 64 K-rows x 64 columns
 constexpr int kBBytes = 4 * kBBox;                // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;    // 48 KB
-constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024;
+constexpr int kBoxBytes = 64 * 128;              // a 64-row x 64-column bf16 box
+constexpr int kOutBytes = 8 * kBoxBytes;          // staging: 2 half tiles x (K nope, V) x 2 column boxes
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + kOutBytes + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kThreads = 6 * 32;
 
@@ -103,25 +109,28 @@ __device__ __forceinline__ bool item_tile(const ExpandParams& p, int b, int j, i
   return *t0 < L;
 }
 
-// Pool row of the first token of a 64-token half tile (valid pages only;
-// rows past the sequence read any in-pool row and are never written).
+// Pool row of the first token of a 64-token half tile: 0 for a half past
+// the sequence (read, never written), -1 for a page outside the pool.
 __device__ __forceinline__ int half_row(const KvLayout& ly, int b, int t, int L) {
   if (ly.page_size == 0) return (int)((long long)b * ly.capacity + t);
   const int nb = (L + ly.page_size - 1) / ly.page_size;
   const int blk = t / ly.page_size;
   if (blk >= nb) return 0;
   const int page = ly.block_table[(long long)b * ly.mbps + blk];
-  if (page < 0 || page >= ly.num_pages) return 0;
+  if (page < 0 || page >= ly.num_pages) return -1;
   return page * ly.page_size + (t % ly.page_size);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     expand_tc_kernel(const __grid_constant__ CUtensorMap lat_map, const __grid_constant__ CUtensorMap uk_map,
-                     const __grid_constant__ CUtensorMap uv_map, const ExpandParams p) {
+                     const __grid_constant__ CUtensorMap uv_map, const __grid_constant__ CUtensorMap k_store,
+                     const __grid_constant__ CUtensorMap v_store, const ExpandParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_base_sh;
+  __shared__ int s_bad;                            // an epilogue warp's wait failed: no more TMA stores
+  uint8_t* s_out = smem + kStages * kStageBytes;   // 1024-aligned staging tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -133,6 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&acc_empty[a], 4);
     }
     ptx::mbar_init(&drain, 1);
+    s_bad = 0;
     ptx::fence_barrier_init();
   }
   if (warp == 1) {
@@ -162,8 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int t0, tlo, thi;
         if (!item_tile(p, b, j, &t0, &tlo, &thi, g == 0)) continue;
         // dense form: rows of the dense matrix (a box past its end reads zeros)
-        const int row0 = p.dense_rows > 0 ? t0 : half_row(p.ly, b, t0, thi);
-        const int row1 = p.dense_rows > 0 ? t0 + 64 : half_row(p.ly, b, t0 + 64, thi);
+        const int row0 = p.dense_rows > 0 ? t0 : max(0, half_row(p.ly, b, t0, thi));
+        const int row1 = p.dense_rows > 0 ? t0 + 64 : max(0, half_row(p.ly, b, t0 + 64, thi));
         for (int kc = 0; kc < kR / kKC; ++kc, ++it) {
           const int s = (int)(it % kStages);
           const long long k = it / kStages;
@@ -267,9 +277,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           row = dense_row_target(p, t);
           write = row >= 0;
         } else {
-          row = half_row(p.ly, b, t0 + (r & ~63), thi) + (r & 63);
+          const int hr = half_row(p.ly, b, t0 + (r & ~63), thi);
+          if (hr < 0) {
+            flag_status(p.st, GQLA_DEV_BAD_PAGE);
+            write = false;
+          }
+          row = (long long)hr + (r & 63);
         }
       }
+      // this warp's 32 rows lie in half tile hh; it goes out by TMA stores when
+      // every one of its 64 rows is written (pool form, both output halves)
+      const int hh = r >> 6;
+      const int h_lo = t0 + 64 * hh;
+      const bool tma_half = ok && p.dense_rows == 0 && hf < 0 && h_lo >= tlo && h_lo + 64 <= thi &&
+                            half_row(p.ly, b, h_lo, thi) >= 0;
       if (ok) {
         ptx::tc_fence_after();
         const int ncol = hf < 0 ? kN / 32 : kN / 64;   // 32-column groups in the accumulator
@@ -278,19 +299,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t v[32];
           ptx::tmem_ld32(tl + (uint32_t)(ab * kN + 32 * c), v);
           ptx::tmem_ld_wait();
-          if (write) {
+          uint4 w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            w[e].x = ptx::pack_bf16(__uint_as_float(v[8 * e + 0]), __uint_as_float(v[8 * e + 1]));
+            w[e].y = ptx::pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3]));
+            w[e].z = ptx::pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5]));
+            w[e].w = ptx::pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7]));
+          }
+          if (tma_half) {
+            // box (half, c / 2) of the staging tile, columns 32 (c % 2) .. of it
+            uint8_t* box = s_out + (hh * 4 + c / 2) * kBoxBytes;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              *reinterpret_cast<uint4*>(box + ptx::swz128(r & 63, 4 * (c & 1) + e)) = w[e];
+          } else if (write) {
             const int oc = hf == 1 ? c + kDn / 32 : c;   // column group of [K nope | V]
             bf16* dst = oc < kDn / 32 ? p.kp + row * p.kr.pitch + p.kr.nope_at(g) + 32 * oc
                                       : p.vp + (row * G + g) * kDv + 32 * (oc - kDn / 32);
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint4 w;
-              w.x = ptx::pack_bf16(__uint_as_float(v[e + 0]), __uint_as_float(v[e + 1]));
-              w.y = ptx::pack_bf16(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-              w.z = ptx::pack_bf16(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
-              w.w = ptx::pack_bf16(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
-              *reinterpret_cast<uint4*>(dst + e) = w;
-            }
+            for (int e = 0; e < 4; ++e) *reinterpret_cast<uint4*>(dst + 8 * e) = w[e];
           }
         }
         if (write && hf != 1 && (p.kr.rope_gs != 0 || g == 0)) {   // a shared RoPE key: by group 0
@@ -304,9 +332,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&acc_empty[ab]);
+      // staged half tiles out with TMA stores, then the staging is free again
+      if (!ok && lane == 0) atomicExch(&s_bad, 1);
+      ptx::fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 2 * 32 && !s_bad) {
+        for (int h = 0; h < 2; ++h) {
+          const int lo = t0 + 64 * h;
+          if (!(p.dense_rows == 0 && hf < 0 && lo >= tlo && lo + 64 <= thi)) continue;
+          const int y = half_row(p.ly, b, lo, thi);
+          if (y < 0) continue;                    // a page outside the pool (flagged by its rows)
+          ptx::tma_store_2d(&k_store, s_out + (h * 4 + 0) * kBoxBytes, p.kr.nope_at(g), y);
+          ptx::tma_store_2d(&k_store, s_out + (h * 4 + 1) * kBoxBytes, p.kr.nope_at(g) + 64, y);
+          ptx::tma_store_2d(&v_store, s_out + (h * 4 + 2) * kBoxBytes, g * kDv, y);
+          ptx::tma_store_2d(&v_store, s_out + (h * 4 + 3) * kBoxBytes, g * kDv + 64, y);
+        }
+        ptx::bulk_commit_group();
+        ptx::bulk_wait_group_read();              // the next item may overwrite the staging
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
       ++li;
     }
     if (!ok && lane == 0) flag_status(p.st, GQLA_DEV_TIMEOUT);
+    if (threadIdx.x == 2 * 32) ptx::bulk_wait_group();   // every store has landed before the CTA ends
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -338,6 +386,8 @@ cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, co
       !tmap_bf16_sw128(&uk_map, W_uk, kDn, (long long)d.G * kR, kDn, kKC) ||
       !tmap_bf16_sw128(&uv_map, W_uv, kDv, (long long)d.G * kR, kDv, kKC))
     return cudaErrorInvalidValue;
+  CUtensorMap k_store, v_store;
+  if (!gqa_pool_maps(p, k_pool, v_pool, &k_store, &v_store)) return cudaErrorInvalidValue;
   ExpandParams prm;
   prm.ly = p.ly;
   prm.kp = (bf16*)k_pool;
@@ -358,7 +408,7 @@ cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, co
   if (e != cudaSuccess) return e;
   const long long grid = prm.n_items < num_sms() ? prm.n_items : num_sms();
   if (grid < 1) return cudaSuccess;
-  expand_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(lat_map, uk_map, uv_map, prm);
+  expand_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(lat_map, uk_map, uv_map, k_store, v_store, prm);
   count_launch();
   return cudaGetLastError();
 }
@@ -373,6 +423,8 @@ cudaError_t tc_expand_dense(const Problem& p, const void* rows, void* k_pool, vo
       !tmap_bf16_sw128(&uk_map, W_uk, kDn, (long long)d.G * kR, kDn, kKC) ||
       !tmap_bf16_sw128(&uv_map, W_uv, kDv, (long long)d.G * kR, kDv, kKC))
     return cudaErrorInvalidValue;
+  CUtensorMap k_store, v_store;   // unused by the dense form (its rows are scattered)
+  if (!gqa_pool_maps(p, k_pool, v_pool, &k_store, &v_store)) return cudaErrorInvalidValue;
   ExpandParams prm;
   prm.ly = p.ly;
   prm.kp = (bf16*)k_pool;
@@ -391,7 +443,7 @@ cudaError_t tc_expand_dense(const Problem& p, const void* rows, void* k_pool, vo
   cudaError_t e = ensure_smem_limit((const void*)expand_tc_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long grid = prm.n_items < num_sms() ? prm.n_items : num_sms();
-  expand_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(lat_map, uk_map, uv_map, prm);
+  expand_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(lat_map, uk_map, uv_map, k_store, v_store, prm);
   count_launch();
   return cudaGetLastError();
 }
