@@ -113,6 +113,24 @@ def test_expand_tail_only_touches_new_tokens():
         assert bool((kp2[b, :L - 2] == sentinel).all()) and bool((vp2[b, L:] == sentinel).all())
 
 
+def test_expand_flags_bad_page_and_writes_nothing_for_it():
+    """A block-table entry outside the pool: flagged, and no row is written in
+    its place; every other page is expanded as without it."""
+    from latent_kv_cache_flash_b200 import gqla
+    d = synth.Dims(**LLAMA)
+    inp = _wl(d, 2, [300, 200], page=64, seed=12)
+    kp_ref, vp_ref = H.run_expand(inp)
+    replaced = int(inp.block_table[1, 1])
+    inp.block_table[1, 1] = inp.num_pages + 3
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    kp, vp = H.run_expand(inp, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & gqla.DEV_BAD_PAGE
+    others = [pg for pg in range(inp.num_pages) if pg != replaced]
+    assert torch.equal(kp[others], kp_ref[others]) and torch.equal(vp[others], vp_ref[others])
+    assert not bool(kp[replaced].any()) and not bool(vp[replaced].any())
+
+
 # ---- combine ------------------------------------------------------------
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_combine_matches_oracle(dtype):
