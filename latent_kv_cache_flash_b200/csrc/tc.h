@@ -18,9 +18,10 @@ bool gqa_pool_maps(const Problem& p, const void* k_pool, const void* v_pool, CUt
 // GQA decode over the expanded cache: mma.sync bf16 tiles, cp.async.bulk
 // staged K/V pages, online softmax per 16-row block.
 bool tc_gqa_supports(const Problem& p);
-// With split partials (o_part) and a counter array of B * G * ceil(m s_q / 16)
-// ints, the mma.sync kernel merges the splits itself into out_final /
-// lse_final and sets *merged; otherwise the caller runs the combine.
+// With split partials (o_part), a counter array of B * G * ceil(m s_q / 16)
+// ints and few rows per group, the mma.sync kernel merges the splits itself
+// into out_final / lse_final and sets *merged; otherwise the caller runs the
+// combine.
 cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, const void* v_pool, void* out,
                           float* o_part, float* lse_dst, int32_t* st, cudaStream_t s, int* counters = nullptr,
                           void* out_final = nullptr, float* lse_final = nullptr, bool* merged = nullptr);

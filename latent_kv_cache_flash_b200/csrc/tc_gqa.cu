@@ -18,10 +18,10 @@
 //    keep an online softmax (running max in the log2 domain) per row;
 //  * the warps' partial states are merged through shared memory at the end;
 //    the result goes to `out` (one split) or to fp32 split partials.  With
-//    split partials, the last CTA of a (sequence, group, row block) to finish
-//    (an atomic count per block) merges all splits' partials by their
-//    log-sum-exp and writes the final output, so no separate combine pass
-//    re-reads them.
+//    split partials and few rows per group (m * s_q * splits <= 64), the last
+//    CTA of a (sequence, group, row block) to finish (an atomic count per
+//    block) merges all splits' partials by their log-sum-exp and writes the
+//    final output, so no separate combine pass re-reads them.
 #include <math.h>
 
 #include "ptx.cuh"
@@ -340,33 +340,55 @@ __global__ void __launch_bounds__(kThreads, 2)
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
     if (last_cta) {
       __threadfence();
-      for (int idx = tid; idx < p.rbc * 16 * (kDv / 4); idx += kConsumerWarps * 32) {
-        const int rl = idx / (kDv / 4), d4 = (idx % (kDv / 4)) * 4;
+      // the ring is idle now: per row of this CTA, the splits' weights
+      const int nrow = min(p.rbc * 16, p.rows_unit - rb0 * 16);
+      float* wtab = reinterpret_cast<float*>(smem);   // [nrow][S]
+      float* rmax = wtab + nrow * S;                  // [nrow]
+      float* rsum = rmax + nrow;                      // [nrow]
+      for (int rl = warp; rl < nrow; rl += kConsumerWarps) {
         const int r = rb0 * 16 + rl;
-        if (r >= p.rows_unit) continue;
         const int i = r / p.m, h = g * p.m + r % p.m;
         const long long gr = ((long long)b * p.s_q + i) * p.n_h + h;
         float mx = -INFINITY;
-        for (int sp = 0; sp < S; ++sp) mx = fmaxf(mx, __ldcg(p.lse + (long long)sp * p.rows + gr));
+        for (int sp = lane; sp < S; sp += 32) mx = fmaxf(mx, __ldcg(p.lse + (long long)sp * p.rows + gr));
+        mx = warp_max(mx);
         float z = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (mx != -INFINITY) {
-          for (int sp = 0; sp < S; ++sp) {
-            const float ls = __ldcg(p.lse + (long long)sp * p.rows + gr);
-            if (ls == -INFINITY) continue;
-            const float w = expf(ls - mx);
-            z += w;
-            const float4 o = __ldcg(reinterpret_cast<const float4*>(p.o_part + ((long long)sp * p.rows + gr) * kDv + d4));
-            acc.x = fmaf(w, o.x, acc.x);
-            acc.y = fmaf(w, o.y, acc.y);
-            acc.z = fmaf(w, o.z, acc.z);
-            acc.w = fmaf(w, o.w, acc.w);
-          }
+        for (int sp = lane; sp < S; sp += 32) {
+          const float ls = __ldcg(p.lse + (long long)sp * p.rows + gr);
+          const float w = (ls == -INFINITY) ? 0.f : expf(ls - mx);
+          wtab[rl * S + sp] = w;
+          z += w;
         }
+        z = warp_sum(z);
+        if (lane == 0) {
+          rmax[rl] = mx;
+          rsum[rl] = z;
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+      // weighted sums: the splits' loads are independent (an empty split holds zeros)
+      for (int idx = tid; idx < nrow * (kDv / 4); idx += kConsumerWarps * 32) {
+        const int rl = idx / (kDv / 4), d4 = (idx % (kDv / 4)) * 4;
+        const int r = rb0 * 16 + rl;
+        const int i = r / p.m, h = g * p.m + r % p.m;
+        const long long gr = ((long long)b * p.s_q + i) * p.n_h + h;
+        const float* src = p.o_part + gr * kDv + d4;
+        const long long sstride = p.rows * kDv;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int sp = 0; sp < S; ++sp) {
+          const float w = wtab[rl * S + sp];
+          const float4 o = __ldcg(reinterpret_cast<const float4*>(src + sp * sstride));
+          acc.x = fmaf(w, o.x, acc.x);
+          acc.y = fmaf(w, o.y, acc.y);
+          acc.z = fmaf(w, o.z, acc.z);
+          acc.w = fmaf(w, o.w, acc.w);
+        }
+        const float z = rsum[rl];
         const float inv = z > 0.f ? 1.f / z : 0.f;
         *reinterpret_cast<uint2*>(p.out_final + gr * kDv + d4) =
             make_uint2(ptx::pack_bf16(acc.x * inv, acc.y * inv), ptx::pack_bf16(acc.z * inv, acc.w * inv));
-        if (d4 == 0 && p.lse_final) p.lse_final[gr] = mx == -INFINITY ? -INFINITY : mx + logf(z);
+        if (d4 == 0 && p.lse_final) p.lse_final[gr] = rmax[rl] == -INFINITY ? -INFINITY : rmax[rl] + logf(z);
       }
       if (tid == 0) *counter = 0;                 // back to zero for the next call
     }
@@ -411,7 +433,10 @@ cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, c
   prm.st = st;
   prm.kr = p.kr;
   dim3 grid(p.plan.num_splits, p.ly.batch * d.G, (rb + prm.rbc - 1) / prm.rbc);
-  const bool merge = o_part && counters && out_final;
+  // Merging in the last CTA pays when a block's merge is small (measured: it
+  // wins at 4 rows x 8 splits, loses at 16-32 rows x 8-16 splits, where the
+  // combine pass spreads the same work over the whole GPU).
+  const bool merge = o_part && counters && out_final && (long long)p.m * d.s_q * p.plan.num_splits <= 64;
   prm.counters = merge ? counters : nullptr;
   prm.out_final = (__nv_bfloat16*)out_final;
   prm.lse_final = lse_final;
