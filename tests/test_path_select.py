@@ -15,13 +15,13 @@ B200 = (148, 6559.0, 1656.2)   # SMs, copy GB/s, dense bf16 TFLOP/s (measured on
 # d = v = 128, B32, L 32K), measured on one B200 with `bench.py --sweep
 # crossover` (absorb ms, GQA ms).  A performance record, not an oracle value.
 MEASURED_B200 = {
-    (1, 1): (0.525, 0.179), (1, 2): (1.005, 0.337), (1, 4): (1.880, 0.632),
-    (2, 1): (0.526, 0.312), (2, 2): (1.005, 0.331), (2, 4): (1.883, 0.631),
-    (4, 1): (0.524, 0.483), (4, 2): (1.005, 0.593), (4, 4): (1.882, 0.632),
-    (8, 1): (0.535, 0.779), (8, 2): (1.010, 0.846), (8, 4): (1.906, 1.110),
-    (16, 1): (0.545, 1.476), (16, 2): (1.006, 1.491), (16, 4): (1.883, 1.593),
-    (32, 1): (0.531, 3.183), (32, 2): (1.007, 2.936), (32, 4): (1.893, 2.950),
-    (128, 1): (0.526, 12.795), (128, 2): (1.008, 12.360), (128, 4): (1.884, 12.420),
+    (1, 1): (0.527, 0.180), (1, 2): (1.005, 0.338), (1, 4): (1.880, 0.632),
+    (2, 1): (0.524, 0.312), (2, 2): (1.004, 0.333), (2, 4): (1.882, 0.630),
+    (4, 1): (0.524, 0.481), (4, 2): (1.004, 0.593), (4, 4): (1.891, 0.632),
+    (8, 1): (0.540, 0.777), (8, 2): (1.009, 0.849), (8, 4): (1.884, 1.106),
+    (16, 1): (0.526, 1.481), (16, 2): (1.003, 1.505), (16, 4): (1.881, 1.600),
+    (32, 1): (0.525, 3.152), (32, 2): (1.004, 2.946), (32, 4): (1.897, 2.976),
+    (128, 1): (0.525, 12.631), (128, 2): (1.009, 12.295), (128, 4): (1.883, 12.372),
 }
 
 
