@@ -36,7 +36,8 @@
  *      q       [B, s_q, n_h, d_nope + d_rope]       nope part first
  *      latent  token rows [c_KV (r) ; k_rope (d_rope)]
  *      K pool  token rows [G, d_nope + d_rope]      (per-group key with its own
- *                                                     copy of k_rope)
+ *                                                     copy of k_rope), or
+ *              [G * d_nope + d_rope] with dims.k_layout = GQLA_K_SHARED_ROPE
  *      V pool  token rows [G, d_v]
  *      W_uk    [G, r, d_nope]      W_uv [G, r, d_v]
  *      out     [B, s_q, n_h, d_v]  lse [B, s_q, n_h]
