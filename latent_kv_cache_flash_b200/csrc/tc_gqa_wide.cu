@@ -241,19 +241,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = ptx::mbar_wait(&s_full[gp], (j >> 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
       // the row maximum over the tile's 64 scores, read in two halves; S[gp]
-      // is next written for tile j + 2, this group's own next tile
+      // is next written for tile j + 2, this group's own next tile.  A tile
+      // that every row of the CTA sees whole needs no mask, and the scale is
+      // applied once to the extreme score (the largest for a positive scale,
+      // the smallest for a negative one).
+      const bool whole = __all_sync(0xffffffffu, !valid || t0 + kT <= vis);
+      const float sgn = p.scale_log2 < 0.f ? -1.f : 1.f;
       float mx = -INFINITY;
       if (ok) {
         ptx::tc_fence_after();
+        float raw = -INFINITY;                    // max of sgn * s over the visible tokens
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t sv[32];
           ptx::tmem_ld32(tl + kSCol + (uint32_t)kT * gp + 32u * h, sv);
           ptx::tmem_ld_wait();
+          if (whole) {
 #pragma unroll
-          for (int t = 0; t < 32; ++t)
-            if (t0 + 32 * h + t < vis) mx = fmaxf(mx, __uint_as_float(sv[t]) * p.scale_log2);
+            for (int t = 0; t < 32; ++t) raw = fmaxf(raw, sgn * __uint_as_float(sv[t]));
+          } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+              if (t0 + 32 * h + t < vis) raw = fmaxf(raw, sgn * __uint_as_float(sv[t]));
+          }
         }
+        mx = (valid && raw != -INFINITY) ? raw * (sgn * p.scale_log2) : -INFINITY;
       }
       float factor = 1.f;
       int need = 0;
@@ -297,10 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&s_free[gp]);
         }
+        // 2^(s * scale - m): one fused multiply-add per score
+        const float neg_m = -m_used;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const float x = (ok && t0 + 32 * h + t < vis) ? __uint_as_float(sv[t]) * p.scale_log2 : -INFINITY;
-          const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(x - m_used);
+          const bool seen = ok && m_used != -INFINITY && (whole || t0 + 32 * h + t < vis);
+          const float e = seen ? ptx::fast_exp2(fmaf(__uint_as_float(sv[t]), p.scale_log2, neg_m)) : 0.f;
           sv[t] = __float_as_uint(e);
           acc += e;
         }

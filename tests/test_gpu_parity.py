@@ -369,3 +369,16 @@ def test_gqa_wide_growing_scores(G, s_q, splits):
         inp.latent[b] = rows.to(inp.latent.dtype)
     out, lse = H.run_decode(inp, "gqa", num_splits=splits)
     H.check_units(inp, out, lse, H.all_units(inp), "gqa wide growing G=%d s_q=%d S=%d" % (G, s_q, splits))
+
+
+@pytest.mark.parametrize("G,s_q", [(1, 2), (8, 1)])
+def test_negative_and_tiny_scales(G, s_q):
+    """The softmax scale is any finite number: a negative one flips which
+    score is largest (the tcgen05 GQA kernel scales the extreme raw score),
+    and a tiny one gives near-uniform weights."""
+    for scale in (-0.09, 1e-4):
+        d = synth.Dims(n_h=128, G=G, d_nope=128, d_rope=64, d_v=128, r=512, s_q=s_q, scale=scale)
+        inp = _wl(d, 2, [700, 131], page=64, seed=77)
+        for path in ("absorb", "gqa"):
+            out, lse = H.run_decode(inp, path)
+            H.check_units(inp, out, lse, H.sample_units(inp, 4, seed=G), "scale %g %s G=%d" % (scale, path, G))
