@@ -272,14 +272,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       float factor = 1.f;
       int need = 0;
       if (ok) {
-        float mx = -INFINITY;
+        // A tile every row of the warp sees whole needs no mask; the scale is
+        // applied once, to the extreme raw score (the largest for a positive
+        // scale, the smallest for a negative one), and the exponent is one
+        // fused multiply-add.
+        const bool whole = __all_sync(0xffffffffu, !valid || t0 + kTk <= vis);
+        const float sgn = p.scale_log2 < 0.f ? -1.f : 1.f;
+        float raw = -INFINITY;                   // max of sgn * s over the visible tokens
+        if (whole) {
 #pragma unroll
-        for (int v = 0; v < kTk / 2; ++v) {
-          const float x = (t0 + 2 * v + half < vis) ? __uint_as_float(sv[v]) * p.scale_log2 : -INFINITY;
-          sv[v] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+          for (int v = 0; v < kTk / 2; ++v) raw = fmaxf(raw, sgn * __uint_as_float(sv[v]));
+        } else {
+#pragma unroll
+          for (int v = 0; v < kTk / 2; ++v)
+            if (t0 + 2 * v + half < vis) raw = fmaxf(raw, sgn * __uint_as_float(sv[v]));
         }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));   // the row's other half
+        raw = fmaxf(raw, __shfl_xor_sync(0xffffffffu, raw, 2));   // the row's other half
+        const float mx = (valid && raw != -INFINITY) ? raw * (sgn * p.scale_log2) : -INFINITY;
         if (m_used == -INFINITY) {
           m_used = mx;                            // O holds only zeros so far
         } else if (mx > m_used + kRescaleLog2) {
@@ -288,10 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_sum *= factor;
           m_used = mx;
         }
+        const float neg_m = -m_used;
         float acc = 0.f;
 #pragma unroll
         for (int v = 0; v < kTk / 2; ++v) {
-          const float e = m_used == -INFINITY ? 0.f : ptx::fast_exp2(__uint_as_float(sv[v]) - m_used);
+          const bool seen = m_used != -INFINITY && (whole || t0 + 2 * v + half < vis);
+          const float e = seen ? ptx::fast_exp2(fmaf(__uint_as_float(sv[v]), p.scale_log2, neg_m)) : 0.f;
           sv[v] = __float_as_uint(e);
           acc += e;
         }

@@ -15,13 +15,13 @@ B200 = (148, 6559.0, 1656.2)   # SMs, copy GB/s, dense bf16 TFLOP/s (measured on
 # d = v = 128, B32, L 32K), measured on one B200 with `bench.py --sweep
 # crossover` (absorb ms, GQA ms).  A performance record, not an oracle value.
 MEASURED_B200 = {
-    (1, 1): (0.527, 0.180), (1, 2): (1.005, 0.338), (1, 4): (1.880, 0.632),
-    (2, 1): (0.524, 0.312), (2, 2): (1.004, 0.333), (2, 4): (1.882, 0.630),
-    (4, 1): (0.524, 0.481), (4, 2): (1.004, 0.593), (4, 4): (1.891, 0.632),
-    (8, 1): (0.540, 0.777), (8, 2): (1.009, 0.849), (8, 4): (1.884, 1.106),
-    (16, 1): (0.526, 1.481), (16, 2): (1.003, 1.505), (16, 4): (1.881, 1.600),
-    (32, 1): (0.525, 3.152), (32, 2): (1.004, 2.946), (32, 4): (1.897, 2.976),
-    (128, 1): (0.525, 12.631), (128, 2): (1.009, 12.295), (128, 4): (1.883, 12.372),
+    (1, 1): (0.505, 0.165), (1, 2): (0.953, 0.312), (1, 4): (1.766, 0.588),
+    (2, 1): (0.504, 0.287), (2, 2): (0.952, 0.309), (2, 4): (1.767, 0.588),
+    (4, 1): (0.503, 0.484), (4, 2): (0.952, 0.538), (4, 4): (1.770, 0.592),
+    (8, 1): (0.504, 0.782), (8, 2): (0.953, 0.854), (8, 4): (1.802, 1.014),
+    (16, 1): (0.509, 1.506), (16, 2): (1.024, 1.531), (16, 4): (1.795, 1.628),
+    (32, 1): (0.507, 3.215), (32, 2): (0.967, 3.001), (32, 4): (1.773, 3.034),
+    (128, 1): (0.510, 13.033), (128, 2): (0.962, 12.660), (128, 4): (1.779, 12.741),
 }
 
 
