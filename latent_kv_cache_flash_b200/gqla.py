@@ -164,6 +164,10 @@ def workspace_for(dims: GqlaDims, layout: GqlaKvLayout, num_splits: int, path: i
 
 def gqla_expand_cache(dims, layout, latent, W_uk, W_uv, k_pool, v_pool, tail_tokens=0, dev_status=None,
                       stream=None):
+    """Expand every cached token (or, with tail_tokens > 0, only each
+    sequence's last tail_tokens) into the per-group pools: K rows
+    [c_KV W_uk^g ; k_rope], V rows c_KV W_uv^g.  Pools share the latent pool's
+    geometry (contiguous or paged through the same block table)."""
     s = lib().gqla_expand_cache(ctypes.byref(dims), ctypes.byref(layout), _ptr(latent), _ptr(W_uk), _ptr(W_uv),
                                 _ptr(k_pool), _ptr(v_pool), int(tail_tokens), _ptr(dev_status),
                                 _stream(stream, latent.device))
@@ -172,6 +176,11 @@ def gqla_expand_cache(dims, layout, latent, W_uk, W_uv, k_pool, v_pool, tail_tok
 
 def gqla_append_tokens(dims, layout, new_rows, latent, W_uk=None, W_uv=None, k_pool=None, v_pool=None,
                        dev_status=None, stream=None):
+    """Write each sequence's s_q new token rows new_rows [B, s_q, r + d_rope]
+    at positions seq_len - s_q .. seq_len - 1: into the latent pool (when
+    latent is given) and, expanded, into the per-group pools (when k_pool and
+    v_pool are given; W_uk and W_uv are then required).  latent=None expands
+    only, reading the rows from new_rows."""
     s = lib().gqla_append_tokens(ctypes.byref(dims), ctypes.byref(layout), _ptr(new_rows), _ptr(latent), _ptr(W_uk),
                                  _ptr(W_uv), _ptr(k_pool), _ptr(v_pool), _ptr(dev_status),
                                  _stream(stream, new_rows.device))
@@ -180,6 +189,11 @@ def gqla_append_tokens(dims, layout, new_rows, latent, W_uk=None, W_uv=None, k_p
 
 def gqla_decode_absorb(dims, layout, q, latent, W_uk, W_uv, out, lse=None, num_splits=0, workspace=None,
                        dev_status=None, stream=None):
+    """Absorb-path decode over the latent pool: q_nope is absorbed into the
+    latent space per group, scores run against [c_KV ; k_rope], the latent
+    output is up-projected by W_uv.  out [B, s_q, n_h, d_v]; lse [B, s_q, n_h]
+    fp32 (natural log) when given.  num_splits 0 takes the library's plan; a
+    workspace of gqla_workspace_bytes is allocated when none is passed."""
     if workspace is None:
         workspace = workspace_for(dims, layout, num_splits, GQLA_PATH_ABSORB, q.device)
     s = lib().gqla_decode_absorb(ctypes.byref(dims), ctypes.byref(layout), _ptr(q), _ptr(latent), _ptr(W_uk),
@@ -191,6 +205,9 @@ def gqla_decode_absorb(dims, layout, q, latent, W_uk, W_uv, out, lse=None, num_s
 
 def gqla_decode_gqa(dims, layout, q, k_pool, v_pool, out, lse=None, num_splits=0, workspace=None,
                     dev_status=None, stream=None):
+    """GQA-path decode over the expanded per-group pools: each group's m heads
+    attend to that group's K/V rows.  Same output, lse, split and workspace
+    conventions as gqla_decode_absorb."""
     if workspace is None:
         workspace = workspace_for(dims, layout, num_splits, GQLA_PATH_GQA, q.device)
     s = lib().gqla_decode_gqa(ctypes.byref(dims), ctypes.byref(layout), _ptr(q), _ptr(k_pool), _ptr(v_pool),
