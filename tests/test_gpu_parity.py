@@ -99,6 +99,43 @@ def test_expand_matches_oracle():
             assert torch.equal(torch.tensor(K[:, g, d.d_nope:]), torch.tensor(rows[:, d.r:]))
 
 
+@pytest.mark.parametrize("lens,page,G", [([100], 0, 8), ([1], 0, 8), ([64, 1, 300], 0, 8), ([64, 1, 300], 64, 8),
+                                         ([129, 257, 1], 64, 16), ([700], 64, 1)])
+def test_expand_odd_tile_counts(lens, page, G):
+    """The whole-cache expansion runs two 128-token tiles per MMA (one per CTA
+    of a pair): an odd tile count, a pair whose second tile lies past its
+    sequence, one-token sequences, G = 1 and G = 16.  Every token's rows
+    against the oracle; the slots past each sequence's end keep the sentinel
+    the pools were filled with."""
+    d = synth.Dims(**dict(LLAMA, G=G))
+    inp = _wl(d, len(lens), lens, page=page, seed=21)
+    ks, vs = synth.expanded_pool_shapes(inp)
+    sentinel = 5.0
+    kp = torch.full(ks, sentinel, dtype=d.torch_dtype, device=DEV)
+    vp = torch.full(vs, sentinel, dtype=d.torch_dtype, device=DEV)
+    H.run_expand(inp, pools=(kp, vp))
+    torch.cuda.synchronize()
+    W_uk = inp.W_uk.double().cpu().numpy()
+    W_uv = inp.W_uv.double().cpu().numpy()
+    for b, L in enumerate(lens):
+        rows = inp.logical_latent(b).double().cpu().numpy()
+        if page:
+            nb = (L + page - 1) // page
+            pages = inp.block_table[b, :nb].long()
+            K = kp[pages].reshape(nb * page, d.G, d.d_qk)
+            V = vp[pages].reshape(nb * page, d.G, d.d_v)
+        else:
+            K, V = kp[b], vp[b]
+        assert bool((K[L:] == sentinel).all()) and bool((V[L:] == sentinel).all()), "written past the end, b=%d" % b
+        K = K[:L].double().cpu().numpy()
+        V = V[:L].double().cpu().numpy()
+        for g in range(d.G):
+            Kr, Vr = O.expand_group(rows[:, : d.r], rows[:, d.r:], W_uk[g], W_uv[g])
+            H.assert_close(K[:, g], Kr, "bf16", "K b=%d g=%d" % (b, g))
+            H.assert_close(V[:, g], Vr, "bf16", "V b=%d g=%d" % (b, g))
+            assert torch.equal(torch.tensor(K[:, g, d.d_nope:]), torch.tensor(rows[:, d.r:]))
+
+
 def test_expand_tail_only_touches_new_tokens():
     d = synth.Dims(**LLAMA, s_q=2)
     inp = _wl(d, 2, [300, 41], seed=5)
