@@ -58,9 +58,19 @@ KvLayout to_kernel_layout(const gqla_kv_layout* l) {
 size_t esize(gqla_dtype t) { return t == GQLA_F32 ? 4 : 2; }
 
 // Split-KV plan.  A requested count is honoured up to rounding the chunk to
-// the kernel's tile.  The automatic choice minimises a simple cost model:
-// (waves of CTAs) x (chunk tokens) x (bytes a CTA streams per token), i.e.
-// the busiest SM's traffic, plus the split partials written and read back.
+// the kernel's tile.  The automatic choice:
+//  * the streaming GQA kernel (two CTAs per SM, HBM-bound): a wave of n CTAs
+//    streams its chunks in the time HBM takes for max(n, ~1.35 per SM) of
+//    them, since fewer CTAs do not keep HBM busy; the plan minimises that
+//    over the waves plus the split partials (B200, LLaMA-shaped layer, B32
+//    L8K: 256 CTAs, one split 0.193 ms, eight 0.218 ms; n_h 128, G 16, B64
+//    L32K: one split leaves a last wave of 136 CTAs, 3.26 ms, two 3.08 ms);
+//  * the tensor-core kernels (one CTA per SM) minimise (waves of CTAs) x
+//    (chunk tokens + the CTA's fixed cost in tokens) x (bytes a CTA streams
+//    per token), the busiest SM's time, plus the split partials written and
+//    read back.  The absorb CTA's prologue and epilogue cost about as much as
+//    300 tokens of its stream (B32 L8K: four splits 0.100 ms, nine 0.112 ms;
+//    B64 L32K, n_h 128: eight splits best).
 SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, gqla_path path, bool tc) {
   const long long L = l.max_seq_len;
   const int granule = !tc ? kSplitGranule : 64;
@@ -74,27 +84,51 @@ SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, 
     return SplitPlan{(int)((L + c - 1) / c), (int)c};
   }
   const long long rows = (long long)l.batch * d.s_q * d.n_h;
+  long long max_s = (L + granule - 1) / granule;
+  if (max_s > kMaxSplits) max_s = kMaxSplits;
+  auto plan_of = [&](long long S) {
+    const long long c = chunk_for(S);
+    return SplitPlan{(int)((L + c - 1) / c), (int)c};
+  };
+  const bool wide = (d.n_h / d.G) * d.s_q >= 64 && tc;
+  if (path == GQLA_PATH_GQA && !wide) {
+    const long long units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 63) / 64);
+    const long long slots = (long long)num_sms() * 2;
+    const long long busy = (long long)num_sms() * 27 / 20;   // CTAs that keep HBM busy
+    const double unit_bytes = 2.0 * (d.d_nope + d.d_rope + d.d_v);
+    const double part_bytes = (double)rows * (d.d_v + 1) * 4 * 2;
+    long long best_s = 1;
+    double best = -1.0;
+    for (long long S = 1; S <= max_s; ++S) {
+      const long long c = chunk_for(S);
+      const long long Se = (L + c - 1) / c;
+      if (Se != S) continue;
+      const long long n = units * Se, rem = n % slots;
+      const double width = (double)(n - rem) + (rem ? (double)(rem > busy ? rem : busy) : 0.0);
+      const double cost = width * c * unit_bytes + (Se > 1 ? Se * part_bytes : 0.0);
+      if (best < 0 || cost < best * 0.999) {
+        best = cost;
+        best_s = Se;
+      }
+    }
+    return plan_of(best_s);
+  }
   long long units, slots;
-  double unit_bytes, part_bytes;
+  double unit_bytes, part_bytes, cta_tokens;
   if (path == GQLA_PATH_ABSORB) {
     units = (long long)l.batch * ((d.n_h * d.s_q + 63) / 64);
     slots = (long long)num_sms() * 1;
     unit_bytes = 2.0 * (d.r + d.d_rope);
     part_bytes = (double)rows * (d.r + 1) * 4 * 2;
-  } else if ((d.n_h / d.G) * d.s_q >= 64 && tc) {
+    cta_tokens = 300.0;
+  } else {
     // the tcgen05 GQA kernel: 128-row blocks, one CTA per SM
     units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 127) / 128);
     slots = (long long)num_sms();
     unit_bytes = 2.0 * (d.d_nope + d.d_rope + d.d_v);
     part_bytes = (double)rows * (d.d_v + 1) * 4 * 2;
-  } else {
-    units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 63) / 64);
-    slots = (long long)num_sms() * 2;
-    unit_bytes = 2.0 * (d.d_nope + d.d_rope + d.d_v);
-    part_bytes = (double)rows * (d.d_v + 1) * 4 * 2;
+    cta_tokens = 0.0;
   }
-  long long max_s = (L + granule - 1) / granule;
-  if (max_s > kMaxSplits) max_s = kMaxSplits;
   long long best_s = 1;
   double best = -1.0;
   for (long long S = 1; S <= max_s; ++S) {
@@ -102,14 +136,13 @@ SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, 
     const long long Se = (L + c - 1) / c;
     if (Se != S) continue;
     const long long waves = (units * Se + slots - 1) / slots;
-    const double cost = (double)waves * c * unit_bytes * slots + (Se > 1 ? Se * part_bytes : 0.0);
+    const double cost = (double)waves * (c + cta_tokens) * unit_bytes * slots + (Se > 1 ? Se * part_bytes : 0.0);
     if (best < 0 || cost < best * 0.999) {
       best = cost;
       best_s = Se;
     }
   }
-  const long long c = chunk_for(best_s);
-  return SplitPlan{(int)((L + c - 1) / c), (int)c};
+  return plan_of(best_s);
 }
 
 }  // namespace

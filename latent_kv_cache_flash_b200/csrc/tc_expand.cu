@@ -38,6 +38,8 @@
 // as many CTAs, each loading half the weights.  Every output element is
 // still the same K-ordered sum of bf16 products, so a token's expansion is
 // the same numbers whichever form produced it.
+#include <mutex>
+
 #include "ptx.cuh"
 #include "tc.h"
 
@@ -51,29 +53,18 @@ constexpr int kR = 512, kDn = 128, kDv = 128, kDr = 64, kE = kR + kDr;
 constexpr int kTM = 128;                          // tokens per tile
 constexpr int kN = kDn + kDv;                     // 256 outputs per group
 constexpr int kKC = 64;                           // K per stage
-#ifndef GQLA_EXPAND_STAGES
-#define GQLA_EXPAND_STAGES 4
-#endif
-constexpr int kStages = GQLA_EXPAND_STAGES;
+constexpr int kStages = 4;
 constexpr int kABytes = kTM * 128;                // 16 KB
 constexpr int kBBox = kKC * 128;                  // 8 KB: 64 K-rows x 64 columns
 constexpr int kBBytes = 4 * kBBox;                // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;    // 48 KB
-#ifndef GQLA_EXPAND_SLOTS
-#define GQLA_EXPAND_SLOTS 2
-#endif
-#ifndef GQLA_EXPAND_EPI_WARPS
-#define GQLA_EXPAND_EPI_WARPS 4
-#endif
-constexpr int kEpiWarps = GQLA_EXPAND_EPI_WARPS;  // 4 per column share of the accumulator
-constexpr int kColShares = kEpiWarps / 4;         // warps that share a TMEM lane quarter
-constexpr int kSlots = GQLA_EXPAND_SLOTS;         // staging boxes per epilogue warp
+constexpr int kEpiWarps = 4;                      // one per TMEM lane quarter
+constexpr int kSlots = 2;                         // staging boxes per epilogue warp
 constexpr int kBoxBytes = 32 * 128;              // a 32-row x 64-column bf16 box (one warp's rows)
 constexpr int kOutBytes = kEpiWarps * kSlots * kBoxBytes;   // a ring of kSlots boxes for each epilogue warp
 constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + kOutBytes + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kThreads = (2 + kEpiWarps) * 32;
-static_assert(kEpiWarps % 4 == 0 && (kN / 2) % (64 * kColShares) == 0, "epilogue warps cover the columns");
 static_assert(kSmemBytes <= 227 * 1024, "ring and staging must fit the shared memory of one CTA");
 
 // This thread's bulk-copy groups, all but the newest n, have read their
@@ -281,7 +272,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------- epilogue
     const int qd = warp & 3;                   // TMEM lane quarter
-    const int ch = (warp - 2) >> 2;            // column share of the accumulator
     const int r = 32 * qd + lane;              // tile row = token offset
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     uint8_t* ring = s_out + (warp - 2) * kSlots * kBoxBytes;
@@ -306,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int hr = half_row(p.ly, b, t0 + (r & ~63), thi);
           if (hr < 0) {
-            if (ch == 0) flag_status(p.st, GQLA_DEV_BAD_PAGE);
+            flag_status(p.st, GQLA_DEV_BAD_PAGE);
             write = false;
           }
           row = (long long)hr + (r & 63);
@@ -314,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // RoPE key rows of this warp (a shared key: by group 0): lanes 8i..8i+7
       // take 16 bytes each of row 4k + i; loaded now, stored after the columns
-      const bool rope = ok && ch == kColShares - 1 && hf != 1 && (p.kr.rope_gs != 0 || g == 0);
+      const bool rope = ok && hf != 1 && (p.kr.rope_gs != 0 || g == 0);
       uint4 rv[8];
       bool rw[8];
       long long rrow[8];
@@ -341,13 +331,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int y0 = hr0 + 32 * (qd & 1);
       if (ok) {
         ptx::tc_fence_after();
-        const int ncg = (hf < 0 ? kN : kN / 2) / (64 * kColShares);   // this warp's 64-column groups
+        const int ncg = (hf < 0 ? kN : kN / 2) / 64;   // 64-column groups in the accumulator
 #pragma unroll 1
         for (int c = 0; c < ncg; ++c) {
-          const int ac = ch * ncg + c;                  // 64-column group of the accumulator
           uint32_t v[64];
-          ptx::tmem_ld32(tl + (uint32_t)(ab * kN + 64 * ac), v);
-          ptx::tmem_ld32(tl + (uint32_t)(ab * kN + 64 * ac + 32), v + 32);
+          ptx::tmem_ld32(tl + (uint32_t)(ab * kN + 64 * c), v);
+          ptx::tmem_ld32(tl + (uint32_t)(ab * kN + 64 * c + 32), v + 32);
           ptx::tmem_ld_wait();
           uint4 w[8];
 #pragma unroll
@@ -357,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             w[e].z = ptx::pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5]));
             w[e].w = ptx::pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7]));
           }
-          const int oc = hf == 1 ? ac + kDn / 64 : ac;  // 64-column group of [K nope | V]
+          const int oc = hf == 1 ? c + kDn / 64 : c;    // 64-column group of [K nope | V]
           if (tma_rows) {
             uint8_t* box = ring + (int)(stores % kSlots) * kBoxBytes;
             if (lane == 0) bulk_wait_read_allbut<kSlots - 1>();   // the box's last store has read it
@@ -750,6 +739,7 @@ bool store_maps(const Problem& p, const void* k_pool, const void* v_pool, CUtens
 // Cluster pairs of the pair kernel that can be resident at once on the
 // current device (0: it cannot run, the single-CTA kernel takes the work).
 int pair_slots() {
+  static std::mutex mu;
   static int cached[64];
   static bool known[64];
   int dev = 0;
@@ -757,16 +747,21 @@ int pair_slots() {
     cudaGetLastError();
     return 0;
   }
+  std::lock_guard<std::mutex> lock(mu);
   if (known[dev]) return cached[dev];
   int n = 0;
-  if (ensure_smem_limit((const void*)expand_pair_kernel, (int)kPSmemBytes) == cudaSuccess) {
+  if (ensure_smem_limit((const void*)expand_pair_kernel, (int)kPSmemBytes) != cudaSuccess) {
+    cudaGetLastError();   // clear only the error of this failed query
+  } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
     cfg.blockDim = dim3(kPThreads, 1, 1);
     cfg.dynamicSmemBytes = kPSmemBytes;
-    if (cudaOccupancyMaxActiveClusters(&n, (const void*)expand_pair_kernel, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void*)expand_pair_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
   }
-  cudaGetLastError();
   cached[dev] = n;
   known[dev] = true;
   return n;
