@@ -387,8 +387,10 @@ def run_ours(args):
         # are tuned here: each candidate pair's graph is timed (outside the
         # reported region) and the fastest pair is kept.
         tuned = {}
-        for ca in (0, 1, 2, 4):
-            for cg in (0, 2, 4, 8):
+        plan_a = gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_ABSORB)
+        plan_g = gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_GQA)
+        for ca in [0] + [c for c in (1, 2, 4) if c != plan_a]:
+            for cg in [0] + [c for c in (1, 2, 4, 8) if c != plan_g]:
                 absorb_splits[0], gqa_splits[0] = ca, cg
                 g = capture()
                 tuned[(ca, cg)] = timed(g.replay, 30) / 30

@@ -60,8 +60,9 @@ size_t esize(gqla_dtype t) { return t == GQLA_F32 ? 4 : 2; }
 // Split-KV plan.  A requested count is honoured up to rounding the chunk to
 // the kernel's tile.  The automatic choice:
 //  * the streaming GQA kernel (two CTAs per SM, HBM-bound): a wave of n CTAs
-//    streams its chunks in the time HBM takes for max(n, ~1.35 per SM) of
-//    them, since fewer CTAs do not keep HBM busy; the plan minimises that
+//    streams its chunks in the time HBM takes for max(n, busy) of them, since
+//    fewer CTAs do not keep HBM busy (busy: about 1.35 CTAs per SM up to 16
+//    rows a group, every slot beyond); the plan minimises that
 //    over the waves plus the split partials (B200, LLaMA-shaped layer, B32
 //    L8K: 256 CTAs, one split 0.193 ms, eight 0.218 ms; n_h 128, G 16, B64
 //    L32K: one split leaves a last wave of 136 CTAs, 3.26 ms, two 3.08 ms);
@@ -94,7 +95,10 @@ SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, 
   if (path == GQLA_PATH_GQA && !wide) {
     const long long units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 63) / 64);
     const long long slots = (long long)num_sms() * 2;
-    const long long busy = (long long)num_sms() * 27 / 20;   // CTAs that keep HBM busy
+    // CTAs that keep HBM busy: beyond 16 rows a group a CTA's MMAs slow its
+    // stream (n_h 128, B32 L32K: G 16, s_q 4 takes 1.63 ms with every slot
+    // filled, 1.73 ms with one split)
+    const long long busy = (d.n_h / d.G) * d.s_q <= 16 ? (long long)num_sms() * 27 / 20 : slots;
     const double unit_bytes = 2.0 * (d.d_nope + d.d_rope + d.d_v);
     const double part_bytes = (double)rows * (d.d_v + 1) * 4 * 2;
     long long best_s = 1;

@@ -15,13 +15,13 @@ B200 = (148, 6559.0, 1656.2)   # SMs, copy GB/s, dense bf16 TFLOP/s (measured on
 # d = v = 128, B32, L 32K), measured on one B200 with `bench.py --sweep
 # crossover` (absorb ms, GQA ms).  A performance record, not an oracle value.
 MEASURED_B200 = {
-    (1, 1): (0.505, 0.165), (1, 2): (0.953, 0.312), (1, 4): (1.766, 0.588),
-    (2, 1): (0.504, 0.287), (2, 2): (0.952, 0.309), (2, 4): (1.767, 0.588),
-    (4, 1): (0.503, 0.484), (4, 2): (0.952, 0.538), (4, 4): (1.770, 0.592),
-    (8, 1): (0.504, 0.782), (8, 2): (0.953, 0.854), (8, 4): (1.802, 1.014),
-    (16, 1): (0.509, 1.506), (16, 2): (1.024, 1.531), (16, 4): (1.795, 1.628),
-    (32, 1): (0.507, 3.215), (32, 2): (0.967, 3.001), (32, 4): (1.773, 3.034),
-    (128, 1): (0.510, 13.033), (128, 2): (0.962, 12.660), (128, 4): (1.779, 12.741),
+    (1, 1): (0.511, 0.166), (1, 2): (0.953, 0.311), (1, 4): (1.766, 0.580),
+    (2, 1): (0.507, 0.287), (2, 2): (0.959, 0.309), (2, 4): (1.768, 0.579),
+    (4, 1): (0.512, 0.487), (4, 2): (0.956, 0.536), (4, 4): (1.767, 0.579),
+    (8, 1): (0.509, 0.745), (8, 2): (0.953, 0.849), (8, 4): (1.769, 0.992),
+    (16, 1): (0.522, 1.483), (16, 2): (0.958, 1.483), (16, 4): (1.782, 1.602),
+    (32, 1): (0.514, 2.934), (32, 2): (0.955, 2.948), (32, 4): (1.779, 2.977),
+    (128, 1): (0.506, 11.878), (128, 2): (0.956, 11.874), (128, 4): (1.770, 11.889),
 }
 
 
