@@ -152,3 +152,41 @@ def test_no_cpu_fallback_when_library_missing(tmp_path, monkeypatch):
     monkeypatch.setattr(gqla, "_lib", None)
     with pytest.raises(ImportError):
         gqla.lib()
+
+
+# Split counts of the automatic plan at shapes where every count was timed on
+# one B200 (CUDA events, resident inputs): the plan must land on the measured
+# best or within its run-to-run noise.  Keys: (n_h, G, s_q, B, L); values:
+# (absorb splits, GQA splits) the plan gives, with the measured best and the
+# call times in the comment.  A performance record, not an oracle value.
+MEASURED_PLANS = {
+    (32, 8, 1, 32, 8192): (4, 1),      # absorb best 4 (0.100 ms; 9: 0.112); GQA best 1 (0.191; 8: 0.218)
+    (32, 8, 2, 32, 8192): (4, 1),      # absorb best 4 (0.103); GQA best 1 (0.191; 8: 0.227)
+    (128, 16, 1, 64, 8192): (1, 2),    # absorb best 1 (0.303; 8: 0.367); GQA 1 and 2 within 0.3% (0.766)
+    (128, 16, 1, 64, 32768): (8, 2),   # absorb best 8 (0.97; 1: 1.03); GQA best 2 (2.94; 1: 3.08)
+    (128, 8, 1, 32, 32768): (9, 1),    # absorb 2/9 within noise (0.51-0.52); GQA best 1 (0.745; 8: 0.78)
+}
+
+
+@pytest.mark.parametrize("shape", sorted(MEASURED_PLANS))
+def test_plan_matches_the_measured_best_split_counts(G, shape):
+    from latent_kv_cache_flash_b200 import synth
+    n_h, groups, s_q, B, L = shape
+    d = G.make_dims(synth.Dims(n_h=n_h, G=groups, d_nope=128, d_rope=64, d_v=128, r=512, s_q=s_q))
+    lens = torch.full((B,), L, dtype=torch.int32)
+    lay = G.make_layout(lens, L, 0, L)
+    got = (G.gqla_num_splits(d, lay, 0, G.GQLA_PATH_ABSORB), G.gqla_num_splits(d, lay, 0, G.GQLA_PATH_GQA))
+    assert got == MEASURED_PLANS[shape]
+
+
+def test_plan_splits_small_batches_to_fill_the_gpu(G):
+    from latent_kv_cache_flash_b200 import synth
+    d = G.make_dims(synth.Dims(n_h=32, G=8, d_nope=128, d_rope=64, d_v=128, r=512))
+    for B, L in ((1, 8192), (4, 8192), (8, 32768)):
+        lens = torch.full((B,), L, dtype=torch.int32)
+        lay = G.make_layout(lens, L, 0, L)
+        # GQA: (sequence, group) units x splits reach about one CTA per SM at least
+        assert B * 8 * G.gqla_num_splits(d, lay, 0, G.GQLA_PATH_GQA) >= 148
+        # absorb: a single wave of 64-row blocks, no more CTAs than SMs
+        S = G.gqla_num_splits(d, lay, 0, G.GQLA_PATH_ABSORB)
+        assert S > 1 and B * S <= 148
