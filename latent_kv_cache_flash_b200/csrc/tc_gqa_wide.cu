@@ -256,9 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t sv[32];
           ptx::tmem_ld32(tl + kSCol + (uint32_t)kT * gp + 32u * h, sv);
           ptx::tmem_ld_wait();
-          if (whole) {
+          if (whole && sgn > 0.f) {
 #pragma unroll
-            for (int t = 0; t < 32; ++t) raw = fmaxf(raw, sgn * __uint_as_float(sv[t]));
+            for (int t = 0; t < 32; ++t) raw = fmaxf(raw, __uint_as_float(sv[t]));
+          } else if (whole) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) raw = fmaxf(raw, -__uint_as_float(sv[t]));
           } else {
 #pragma unroll
             for (int t = 0; t < 32; ++t)
@@ -309,14 +312,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&s_free[gp]);
         }
-        // 2^(s * scale - m): one fused multiply-add per score
+        // 2^(s * scale - m): one fused multiply-add per score; a whole tile
+        // needs no per-score mask
         const float neg_m = -m_used;
+        if (ok && whole && m_used != -INFINITY) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const bool seen = ok && m_used != -INFINITY && (whole || t0 + 32 * h + t < vis);
-          const float e = seen ? ptx::fast_exp2(fmaf(__uint_as_float(sv[t]), p.scale_log2, neg_m)) : 0.f;
-          sv[t] = __float_as_uint(e);
-          acc += e;
+          for (int t = 0; t < 32; ++t) {
+            const float e = ptx::fast_exp2(fmaf(__uint_as_float(sv[t]), p.scale_log2, neg_m));
+            sv[t] = __float_as_uint(e);
+            acc += e;
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const bool seen = ok && m_used != -INFINITY && t0 + 32 * h + t < vis;
+            const float e = seen ? ptx::fast_exp2(fmaf(__uint_as_float(sv[t]), p.scale_log2, neg_m)) : 0.f;
+            sv[t] = __float_as_uint(e);
+            acc += e;
+          }
         }
 #pragma unroll
         for (int g8 = 0; g8 < 4; ++g8) {
