@@ -22,7 +22,7 @@ constexpr double kDefaultTcTflops = 1656.2;
 // Efficiencies of the kernels against those two rates (measured over the
 // crossover grid n_h 128, G 1..128, s_q 1..4, B32, L 32K):
 constexpr double kEtaStream = 1.08;     // GQA mma.sync kernel: K/V read stream (1.07..1.10 of the copy rate at G >= 8)
-constexpr double kEtaWideTc = 0.36;     // GQA tcgen05 kernel: softmax-bound 128-row tiles (two warpgroups)
+constexpr double kEtaWideTc = 0.40;     // GQA tcgen05 kernel: softmax-bound 128-row tiles (two warpgroups)
 constexpr double kEtaAbsorbTc = 0.41;   // absorb tcgen05 kernel: M=64 tiles, N=64 score MMAs
 constexpr double kEtaAbsorbBw = 0.90;   // absorb latent stream when the tensor side keeps up
 constexpr double kLaunchUs = 3.0;       // one kernel launch on a busy stream

@@ -15,13 +15,13 @@ B200 = (148, 6559.0, 1656.2)   # SMs, copy GB/s, dense bf16 TFLOP/s (measured on
 # d = v = 128, B32, L 32K), measured on one B200 with `bench.py --sweep
 # crossover` (absorb ms, GQA ms).  A performance record, not an oracle value.
 MEASURED_B200 = {
-    (1, 1): (0.511, 0.166), (1, 2): (0.953, 0.311), (1, 4): (1.766, 0.580),
-    (2, 1): (0.507, 0.287), (2, 2): (0.959, 0.309), (2, 4): (1.768, 0.579),
-    (4, 1): (0.512, 0.487), (4, 2): (0.956, 0.536), (4, 4): (1.767, 0.579),
-    (8, 1): (0.509, 0.745), (8, 2): (0.953, 0.849), (8, 4): (1.769, 0.992),
-    (16, 1): (0.522, 1.483), (16, 2): (0.958, 1.483), (16, 4): (1.782, 1.602),
-    (32, 1): (0.514, 2.934), (32, 2): (0.955, 2.948), (32, 4): (1.779, 2.977),
-    (128, 1): (0.506, 11.878), (128, 2): (0.956, 11.874), (128, 4): (1.770, 11.889),
+    (1, 1): (0.506, 0.151), (1, 2): (0.954, 0.286), (1, 4): (1.768, 0.535),
+    (2, 1): (0.505, 0.275), (2, 2): (0.955, 0.281), (2, 4): (1.770, 0.536),
+    (4, 1): (0.504, 0.489), (4, 2): (0.955, 0.514), (4, 4): (1.770, 0.537),
+    (8, 1): (0.510, 0.759), (8, 2): (0.989, 0.861), (8, 4): (1.841, 0.961),
+    (16, 1): (0.539, 1.512), (16, 2): (0.958, 1.512), (16, 4): (1.800, 1.627),
+    (32, 1): (0.508, 2.987), (32, 2): (0.958, 3.002), (32, 4): (1.776, 3.033),
+    (128, 1): (0.509, 12.192), (128, 2): (0.963, 12.198), (128, 4): (1.777, 12.210),
 }
 
 
