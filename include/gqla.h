@@ -139,7 +139,11 @@ typedef struct gqla_kv_layout {
  *           G*d_nope + d_rope with GQLA_K_SHARED_ROPE (written)
  *   v_pool  device, pool with rows of G*d_v elements (written)
  * All three pools use `layout`.  Rows outside the expanded range are not
- * touched. */
+ * touched.  With the bf16 tensor-core kernels the whole-cache form
+ * (tail_tokens <= 0) launches clusters of two CTAs (one MMA tile over both);
+ * on a device where such pairs cannot be resident it uses one CTA per tile.
+ * Every output element is the same K-ordered sum of bf16 products either
+ * way. */
 gqla_status gqla_expand_cache(const gqla_dims* dims, const gqla_kv_layout* layout,
                               const void* latent, const void* W_uk, const void* W_uv,
                               void* k_pool, void* v_pool, int32_t tail_tokens,
