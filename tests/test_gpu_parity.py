@@ -136,6 +136,37 @@ def test_expand_odd_tile_counts(lens, page, G):
             assert torch.equal(torch.tensor(K[:, g, d.d_nope:]), torch.tensor(rows[:, d.r:]))
 
 
+@pytest.mark.parametrize("page", [0, 64])
+def test_expand_flags_bad_sequences_and_skips_them(page):
+    """Whole-cache expansion with an empty sequence and one longer than the
+    host bound: both flagged, their slots keep the sentinel, and the healthy
+    sequence's rows equal an expansion without the bad ones, bit for bit."""
+    from latent_kv_cache_flash_b200 import gqla
+    d = synth.Dims(**LLAMA)
+    inp = _wl(d, 3, [200, 300, 150], page=page, seed=14)
+    kp_ref, vp_ref = H.run_expand(inp)
+    ks, vs = synth.expanded_pool_shapes(inp)
+    kp = torch.full(ks, 5.0, dtype=d.torch_dtype, device=DEV)
+    vp = torch.full(vs, 5.0, dtype=d.torch_dtype, device=DEV)
+    inp.seq_lens[0] = 0                       # empty
+    inp.seq_lens[2] = 400                     # above the host bound max_seq_len = 300
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    H.run_expand(inp, dev_status=st, pools=(kp, vp))
+    torch.cuda.synchronize()
+    flags = int(st.item())
+    assert flags & gqla.DEV_SHORT_SEQ and flags & gqla.DEV_OVERFLOW
+    if page:
+        rows = lambda b: inp.block_table[b, : (inp.seq_lens_host[b] + 63) // 64].long()
+        for b in (0, 2):
+            assert bool((kp[rows(b)] == 5.0).all()) and bool((vp[rows(b)] == 5.0).all())
+        flat = lambda t: t[rows(1)].reshape((-1,) + tuple(t.shape[2:]))[:300]
+        assert torch.equal(flat(kp), flat(kp_ref)) and torch.equal(flat(vp), flat(vp_ref))
+    else:
+        for b in (0, 2):
+            assert bool((kp[b] == 5.0).all()) and bool((vp[b] == 5.0).all())
+        assert torch.equal(kp[1, :300], kp_ref[1, :300]) and torch.equal(vp[1, :300], vp_ref[1, :300])
+
+
 def test_expand_tail_only_touches_new_tokens():
     d = synth.Dims(**LLAMA, s_q=2)
     inp = _wl(d, 2, [300, 41], seed=5)
