@@ -410,7 +410,7 @@ def run_ours(args):
     ms_append = timed(append_latent, reps) / reps
     ms_append_expand = timed(append, reps) / reps
     ms_expand_full = timed(lambda: gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0,
-                                                          status), 3) / 3
+                                                          status), 10) / 10
     # the GQA call over the same cache with the RoPE key stored once per token
     # row (a second, smaller K pool; V is shared)
     dims_s = gqla.make_dims(dataclasses.replace(d, k_shared_rope=True))
