@@ -1,19 +1,27 @@
 """GQLA decode-attention benchmark (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--sq 1|2] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dsv3_64k|llama3_8b] [--sq 1|2]
+                    [--impl ours|reference] [--sweep crossover|context|ragged|capacity]
 
-Workload: the LLaMA-3-8B-shaped GQLA layer (n_h 32, G 8, d_nope 128, d_rope
-64, d_v 128, r 512), batch 32, uniform context 8192, s_q new tokens per
-sequence, bf16, synthetic seeded inputs.  One step is one pass of the whole
-decode hot path over that batch: the decode-time expansion of the s_q new
-tokens into the per-group cache, the MQA-absorb decode and the GQA decode
-(both paths produce the batch's B*s_q output tokens).  value = decoded tokens
-(B*s_q per step, per GPU) / device time.  Under torchrun every rank decodes
-its own batch (weak scaling; sequences are independent, no data-path
-collective); the time is the max over ranks.
+Default workload: the DeepSeek-V3-shaped GQLA layer (n_h 128, G 16, d_nope
+128, d_rope 64, d_v 128, r 512), batch 64, uniform context 65536, s_q new
+tokens per sequence, bf16, synthetic seeded inputs: the largest single-GPU
+configuration of the decode study.  --workload llama3_8b selects the
+LLaMA-3-8B-shaped layer (n_h 32, G 8), batch 32, context 8192.
+
+One step is one decode step of that batch: the s_q new tokens' latent rows
+are written into the latent pool, their expansion is written into the
+per-group pools (which the GQA path reads and a runtime keeps current so it
+can switch paths), and the decode path the library's selector picks for the
+workload runs over the whole cache (append, expansion, decode: the hot path
+of one step).  The other path is timed on the same inputs and reported under
+"paths".  value = decoded tokens (B*s_q per step per GPU) / device time.
+Under torchrun every rank decodes its own batch (weak scaling; sequences are
+independent, no data-path collective); the time is the max over ranks.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this build)
-on the same workload, one bounded sample of (sequence, group) units per step.
+on the same workload: each step decodes one (sequence, group) unit of the
+batch, and its rate is scaled by the batch's number of such units.
 """
 from __future__ import annotations
 
@@ -26,12 +34,14 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode attention tokens/s per layer and % of roofline (HBM GB/s or TC util), 1×B200"
+WORKLOADS = ("dsv3_64k", "llama3_8b")
 
 
 def load_peaks():
@@ -45,40 +55,81 @@ def load_peaks():
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="dsv3_64k", choices=WORKLOADS)
     ap.add_argument("--sq", type=int, default=1, choices=[1, 2])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", choices=["select", "absorb", "gqa"], default="select",
+                    help="decode path of the step: the library's selector (default) or a fixed one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
     ap.add_argument("--tp", action="store_true",
                     help="with --gpus N > 1: split the groups of one batch over the ranks (strong scaling) "
                          "instead of giving every rank its own batch")
+    ap.add_argument("--once", choices=["absorb", "gqa"],
+                    help="profiling case: build a DeepSeek-V3-shaped batch of --batch sequences of --seq-len "
+                         "tokens with --groups groups, run --warmup calls of this path, then one more, and exit")
+    ap.add_argument("--batch", type=int, default=8)
+    ap.add_argument("--seq-len", type=int, default=8192)
+    ap.add_argument("--groups", type=int, default=16)
     ap.add_argument("--sweep", choices=["crossover", "context", "ragged", "capacity"],
                     help="instead of the headline line, time both decode paths over a workload sweep "
                          "(one JSON line per point)")
     return ap.parse_args()
 
 
-def workload(s_q):
+def workload(name, s_q):
     from latent_kv_cache_flash_b200 import synth
-    return synth.llama3_8b(s_q=s_q)
+    if name == "llama3_8b":
+        return synth.llama3_8b(s_q=s_q)
+    return synth.dsv3(seq_len=65536, s_q=s_q)
+
+
+def bench_config(wl, world=1, tp=False):
+    """The workload's description, the same dict in both arms of the bench."""
+    d = wl.dims
+    T = wl.batch * wl.seq_len
+    return {"workload": "%s B%d L%d s_q%d" % (wl.name, wl.batch, wl.seq_len, d.s_q), "batch": wl.batch,
+            "seq_len": wl.seq_len, "s_q": d.s_q, "n_h": d.n_h, "G": d.G, "d_nope": d.d_nope,
+            "d_rope": d.d_rope, "d_v": d.d_v, "r": d.r, "dtype": d.dtype,
+            "l2": "no flush: inputs larger than L2 (latent cache %.0f MB, expanded cache %.0f MB)" % (
+                2 * T * (d.r + d.d_rope) / 1e6, 2 * T * d.G * (d.d_qk + d.d_v) / 1e6),
+            "parallelism": ("tp%d over groups (each rank: G/%d groups and their heads; no collective inside "
+                            "attention)" % (world, world)) if tp else
+                           "replicas x%d (batch-sharded, no collective)" % world}
 
 
 def algorithmic(wl):
-    """Per-step algorithmic bytes and flops of each path (the method's own
-    traffic: cache bytes read once per step, q/out/weights ignored)."""
+    """Per-step algorithmic bytes and flops (the method's own traffic: every
+    cached byte a path reads once per step; q, out and weights ignored) of
+    each decode path, of the new tokens' append and expansion, and of the
+    whole-cache expansion."""
     d = wl.dims
-    T = wl.batch * wl.seq_len
-    keys = sum(wl.seq_len - d.s_q + i + 1 for i in range(d.s_q)) * wl.batch   # (query, key) pairs per head
-    absorb_bytes = 2 * T * (d.r + d.d_rope)
-    absorb_flops = d.n_h * keys * 2 * (2 * d.r + d.d_rope) + wl.batch * d.s_q * d.n_h * 2 * d.r * (d.d_nope + d.d_v)
-    gqa_bytes = 2 * T * d.G * (d.d_qk + d.d_v)
-    gqa_flops = d.n_h * keys * 2 * (d.d_qk + d.d_v)
-    gqa_shared_bytes = 2 * T * (d.G * (d.d_nope + d.d_v) + d.d_rope)
-    return dict(absorb_bytes=absorb_bytes, absorb_flops=absorb_flops, gqa_bytes=gqa_bytes, gqa_flops=gqa_flops,
-                gqa_shared_bytes=gqa_shared_bytes)
+    B = wl.batch
+    T = B * wl.seq_len
+    keys = sum(wl.seq_len - d.s_q + i + 1 for i in range(d.s_q)) * B   # (query, key) pairs per head
+    E = d.r + d.d_rope
+    new = B * d.s_q
+    return dict(
+        absorb_bytes=2 * T * E,
+        absorb_flops=d.n_h * keys * 2 * (2 * d.r + d.d_rope) + new * d.n_h * 2 * d.r * (d.d_nope + d.d_v),
+        gqa_bytes=2 * T * d.G * (d.d_qk + d.d_v),
+        gqa_flops=d.n_h * keys * 2 * (d.d_qk + d.d_v),
+        gqa_shared_bytes=2 * T * (d.G * (d.d_nope + d.d_v) + d.d_rope),
+        # new rows written into the latent pool; then read, expanded and written per group
+        append_bytes=2 * new * E,
+        expand_new_bytes=2 * new * E + 2 * new * d.G * (d.d_qk + d.d_v),
+        expand_new_flops=2 * new * d.r * d.G * (d.d_nope + d.d_v),
+        expand_full_bytes=2 * T * E + 2 * T * d.G * (d.d_qk + d.d_v),
+        expand_full_flops=2 * T * d.r * d.G * (d.d_nope + d.d_v))
+
+
+def roof_time(nbytes, flops, hbm, tf):
+    """Roofline time (s) and its binding resource."""
+    t_hbm, t_tc = nbytes / (hbm * 1e9), flops / (tf * 1e12)
+    return max(t_hbm, t_tc), ("hbm" if t_hbm >= t_tc else "tensor")
 
 
 # ---------------------------------------------------------------- clocks ---
@@ -90,8 +141,8 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.proc = None
         self.idx = gpu_index
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench.csv") if os.path.isdir(
-            os.path.join(ROOT, "gpurun_out")) else "/tmp/gqla_clocks.csv"
+        fd, self.path = tempfile.mkstemp(prefix="gqla_clocks_", suffix=".csv")
+        os.close(fd)
 
     def start(self):
         try:
@@ -111,7 +162,7 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
-        sm, mx, reasons = [], None, set()
+        sm, power, mx, reasons = [], [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             p = [x.strip() for x in line.split(",")]
@@ -120,32 +171,36 @@ class ClockSampler:
             try:
                 sm.append(float(p[1]))
                 mx = float(p[2])
+                power.append(float(p[3]))
             except ValueError:
                 continue
             for n, v in zip(names, p[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
 
 
 # --------------------------------------------------------- cpu baseline ---
-def oracle_sample(inp, units, both_forms=True):
-    """Runs the oracle on (sequence, group) units; returns seconds."""
-    import numpy as np
+def oracle_unit(inp, unit):
+    """The oracle's decode of one (sequence, group) unit in the expanded form
+    (the definition); returns seconds."""
     from oracle import gqla_oracle as O
     d = inp.dims
+    b, g = unit
     W_uk = inp.W_uk.double().cpu().numpy()
     W_uv = inp.W_uv.double().cpu().numpy()
+    rows = inp.logical_latent(b).double().cpu().numpy()
+    qb = inp.q[b].double().cpu().numpy()
+    L = inp.seq_lens_host[b]
     t0 = time.perf_counter()
-    for b, g in units:
-        rows = inp.logical_latent(b).double().cpu().numpy()
-        qb = inp.q[b].double().cpu().numpy()
-        L = inp.seq_lens_host[b]
-        O.decode_sequence_gqa(qb, rows[:, :d.r], rows[:, d.r:], W_uk, W_uv, L, d.softmax_scale, groups=[g])
-        if both_forms:
-            O.decode_sequence_absorb(qb, rows[:, :d.r], rows[:, d.r:], W_uk, W_uv, L, d.softmax_scale, groups=[g])
+    O.decode_sequence_gqa(qb, rows[:, :d.r], rows[:, d.r:], W_uk, W_uv, L, d.softmax_scale, groups=[g])
     return time.perf_counter() - t0
 
 
@@ -158,52 +213,57 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
+def shuffled_units(wl):
+    import random
+    units = [(b, g) for b in range(wl.batch) for g in range(wl.dims.G)]
+    random.Random(0).shuffle(units)
+    return units
+
+
 def cpu_baseline(inp, budget_s=12.0):
     wl = inp.wl
     d = wl.dims
-    all_units = [(b, g) for b in range(wl.batch) for g in range(d.G)]
-    import random
-    rnd = random.Random(0)
-    rnd.shuffle(all_units)
+    units = shuffled_units(wl)
     done, spent = 0, 0.0
-    while done < len(all_units) and (spent < budget_s or done < 2):
-        spent += oracle_sample(inp, [all_units[done]])
+    while done < len(units) and (spent < budget_s or done < 2):
+        spent += oracle_unit(inp, units[done])
         done += 1
-    per_step = spent / done * len(all_units)
+    per_step = spent / done * len(units)
     return {"value": wl.batch * d.s_q / per_step, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": "%d of %d (sequence, group) units of %s (B%d L%d s_q%d), fp64 expanded and absorb forms, "
-                      "%.1f s, extrapolated linearly to the whole batch" % (
-                          done, len(all_units), wl.name, wl.batch, wl.seq_len, d.s_q, spent)}
+            "sample": "%d of the %d (sequence, group) units of %s (B%d L%d s_q%d) decoded by the fp64 oracle "
+                      "(expanded form, the definition) in %.1f s; the rate is scaled to the whole batch" % (
+                          done, len(units), wl.name, wl.batch, wl.seq_len, d.s_q, spent)}
 
 
 # ----------------------------------------------------------- reference ---
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
-    import torch
     from latent_kv_cache_flash_b200 import synth
-    wl = workload(args.sq)
+    wl = workload(args.workload, args.sq)
     inp = synth.make_inputs(wl, "cpu")
     d = wl.dims
-    all_units = [(b, g) for b in range(wl.batch) for g in range(d.G)]
-    # one unit per step keeps the whole run within a few minutes
+    units = shuffled_units(wl)
     for w in range(args.warmup):
-        oracle_sample(inp, [all_units[w % len(all_units)]])
-    t = 0.0
+        oracle_unit(inp, units[w % len(units)])
+    times = []
     for s in range(args.steps):
-        t += oracle_sample(inp, [all_units[(args.warmup + s) % len(all_units)]])
-    per_unit = t / args.steps
-    step_s = per_unit * len(all_units)
-    value = wl.batch * d.s_q / step_s
+        times.append(oracle_unit(inp, units[(args.warmup + s) % len(units)]))
+    step_s = sum(times) / len(times)
+    # one unit of the B*G per step: the batch's tokens scaled by that share
+    value = wl.batch * d.s_q / len(units) / step_s
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "%s B%d L%d s_q%d" % (wl.name, wl.batch, wl.seq_len, d.s_q), "batch": wl.batch,
-                       "seq_len": wl.seq_len, "s_q": d.s_q, "n_h": d.n_h, "G": d.G, "r": d.r},
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Gaussian, "
+            "random-init weights)", "config": bench_config(wl, world, args.tp),
+            "step": ("one (sequence, group) unit of the batch decoded by the fp64 oracle (expanded form); "
+                     "ms_per_step is that measured time, value scales its rate by the %d units of the batch"
+                     % len(units)),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-                             "sample": "one (sequence, group) unit per step, fp64 expanded and absorb forms, "
-                                       "extrapolated to %d units per step" % len(all_units)},
+                             "sample": "one of the %d (sequence, group) units per step, %d steps, fp64 expanded "
+                                       "form, on rank 0's host cores" % (len(units), args.steps)},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -218,14 +278,15 @@ def kernel_sha(files):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(name):
-    """DRAM bytes per launch from the committed ncu record of this kernel, or
-    None when the kernel's sources changed since the counters were taken."""
+def recorded_traffic(name, workload_name):
+    """DRAM bytes per launch from the committed ncu record of this call on
+    this workload, or None when the kernels' sources changed since the
+    counters were taken (or none were taken)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        rec = json.load(open(p)).get(name)
+        rec = json.load(open(p)).get("%s @ %s" % (name, workload_name))
         if not rec or rec.get("source_sha") != kernel_sha(rec["files"]):
             return None
     except Exception:
@@ -250,8 +311,9 @@ def run_ours(args):
     build.build()
     hbm, tf_burst, tf_sust, peak_src = load_peaks()
 
-    wl = workload(args.sq)
+    wl = workload(args.workload, args.sq)
     tp = args.tp and world > 1
+    config = bench_config(wl, world, tp)
     if not tp:
         wl.seed = multi.rank_seed(wl.seed, rank)   # replicas: every rank its own batch
     inp = synth.make_inputs(wl, dev)
@@ -265,23 +327,10 @@ def run_ours(args):
     kp = torch.empty(ks, dtype=d.torch_dtype, device=dev)
     vp = torch.empty(vs, dtype=d.torch_dtype, device=dev)
     B = wl.batch
-    out_a = torch.empty((B, d.s_q, d.n_h, d.d_v), dtype=d.torch_dtype, device=dev)
-    out_g = torch.empty_like(out_a)
-    lse_a = torch.empty((B, d.s_q, d.n_h), device=dev)
-    lse_g = torch.empty_like(lse_a)
-    # the absorb workspace sized for any split count the step may use
-    ws_a = gqla.workspace_for(dims, lay, 8, gqla.GQLA_PATH_ABSORB, dev)
-    ws_a0 = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_ABSORB, dev)
-    if ws_a0.numel() > ws_a.numel():
-        ws_a = ws_a0
-    del ws_a0
-    absorb_splits = [0]            # 0 = the library's plan for the whole GPU
-    gqa_splits = [0]
-    ws_g = gqla.workspace_for(dims, lay, 8, gqla.GQLA_PATH_GQA, dev)
-    ws_g0 = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_GQA, dev)
-    if ws_g0.numel() > ws_g.numel():
-        ws_g = ws_g0
-    del ws_g0
+    out = torch.empty((B, d.s_q, d.n_h, d.d_v), dtype=d.torch_dtype, device=dev)
+    lse = torch.empty((B, d.s_q, d.n_h), device=dev)
+    ws_a = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_ABSORB, dev)
+    ws_g = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_GQA, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -293,54 +342,35 @@ def run_ours(args):
     Lmax = wl.seq_len
     new_rows = inp.latent[:, Lmax - d.s_q:Lmax].contiguous()
 
+    sel_path, sel_absorb_us, sel_gqa_us = gqla.gqla_select_path(dims, lay, sum(inp.seq_lens_host))
+    if args.path == "absorb":
+        path = gqla.GQLA_PATH_ABSORB
+    elif args.path == "gqa":
+        path = gqla.GQLA_PATH_GQA
+    else:
+        path = sel_path
+    path_name = "absorb" if path == gqla.GQLA_PATH_ABSORB else "gqa"
+
     def append_latent():
         gqla.gqla_append_tokens(dims, lay, new_rows, inp.latent, dev_status=status)
 
-    def append():
-        # the new rows into the latent pool, then their expansion into the per-group pools
-        gqla.gqla_append_tokens(dims, lay, new_rows, inp.latent, inp.W_uk, inp.W_uv, kp, vp, dev_status=status)
-
     def expand_new():
-        # the new rows' expansion alone (no latent pool argument)
+        # the new rows' expansion alone (no latent pool argument): dense rows,
+        # many sequences' new tokens to one 128-row tensor-core tile
         gqla.gqla_append_tokens(dims, lay, new_rows, None, inp.W_uk, inp.W_uv, kp, vp, dev_status=status)
 
-    def expand_tail():
-        gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, d.s_q, status)
-
     def absorb():
-        gqla.gqla_decode_absorb(dims, lay, inp.q, inp.latent, inp.W_uk, inp.W_uv, out_a, lse_a, absorb_splits[0],
-                                ws_a, status)
+        gqla.gqla_decode_absorb(dims, lay, inp.q, inp.latent, inp.W_uk, inp.W_uv, out, lse, 0, ws_a, status)
 
     def gqa():
-        gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out_g, lse_g, gqa_splits[0], ws_g, status)
+        gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out, lse, 0, ws_g, status)
+
+    decode = absorb if path == gqla.GQLA_PATH_ABSORB else gqa
 
     def step():
-        append()
-        absorb()
-        gqa()
-
-    # The two paths of a step share no data once the new tokens are in the
-    # pools: the absorb path runs on a second stream, forked from and joined
-    # back into the main one, so its CTAs and the GQA path's share the machine.
-    side = torch.cuda.Stream(dev)
-
-    def step_overlapped(after_absorb=None, after_gqa=None):
-        main = torch.cuda.current_stream(dev)   # the capture stream while a graph is recorded
-        append_latent()                         # what the absorb path needs ...
-        fork = torch.cuda.Event()
-        fork.record(main)
-        side.wait_event(fork)
-        with torch.cuda.stream(side):
-            absorb()
-            if after_absorb:
-                after_absorb()                  # e.g. its output's copy to the host, on the same stream
-        expand_new()                            # ... and what the GQA path needs, beside the absorb call
-        gqa()
-        if after_gqa:
-            after_gqa()
-        join = torch.cuda.Event()
-        join.record(side)
-        main.wait_event(join)
+        append_latent()
+        expand_new()
+        decode()
 
     barrier = multi.barrier
 
@@ -363,105 +393,106 @@ def run_ours(args):
     if clocks:
         clocks.start()
         time.sleep(0.3)
+
+    # eager timed region: every C-ABI call made on every step; CUDA events
+    # around the decode call of each step (the dominant call) on its stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def eager_steps():
+        for i in range(args.steps):
+            append_latent()
+            expand_new()
+            ev[i][0].record(stream)
+            decode()
+            ev[i][1].record(stream)
+
     n0 = gqla.gqla_launch_counter()
-    eager_ms = timed(step, args.steps) / args.steps
+    eager_ms = timed(eager_steps, 1) / args.steps
     launches = gqla.gqla_launch_counter() - n0
+    ms_decode_live = multi.max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, dev)
+
     # the same step captured once as a CUDA graph and replayed (no host
     # launch gaps between the kernels); every kernel still runs each step
     graph = None
-    tuned = None
     if not args.no_graph:
-        def capture():
-            for _ in range(3):
-                step_overlapped()
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                step_overlapped()
-            for _ in range(3):
-                g.replay()
-            return g
-
-        # The split plan of a call assumes it has the whole GPU; in the
-        # overlapped step the two decode calls share it, so their split counts
-        # are tuned here: each candidate pair's graph is timed (outside the
-        # reported region) and the fastest pair is kept.
-        tuned = {}
-        plan_a = gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_ABSORB)
-        plan_g = gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_GQA)
-        for ca in [0] + [c for c in (1, 2, 4) if c != plan_a]:
-            for cg in [0] + [c for c in (1, 2, 4, 8) if c != plan_g]:
-                absorb_splits[0], gqa_splits[0] = ca, cg
-                g = capture()
-                tuned[(ca, cg)] = timed(g.replay, 30) / 30
-                del g
-        absorb_splits[0], gqa_splits[0] = min(tuned, key=tuned.get)
-        graph = capture()
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
         ms_step = timed(graph.replay, args.steps) / args.steps
     else:
         ms_step = eager_ms
+
     # per-call breakdown (each over at least ~0.3 s of device time)
     reps = args.steps if args.no_clocks else max(args.steps, int(300.0 / max(ms_step, 1e-3)))
-    step_splits = (absorb_splits[0], gqa_splits[0])
-    absorb_splits[0] = gqa_splits[0] = 0   # alone, each call takes the library's own plan
     ms_absorb = timed(absorb, reps) / reps
     ms_gqa = timed(gqa, reps) / reps
-    ms_tail = timed(expand_tail, reps) / reps
     ms_append = timed(append_latent, reps) / reps
-    ms_append_expand = timed(append, reps) / reps
+    ms_expand_new = timed(expand_new, reps) / reps
+    n_full = 5 if wl.seq_len * B > 1 << 20 else 10
     ms_expand_full = timed(lambda: gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0,
-                                                          status), 10) / 10
+                                                          status), n_full) / n_full
     # the GQA call over the same cache with the RoPE key stored once per token
-    # row (a second, smaller K pool; V is shared)
+    # row (a smaller K pool; V is shared); the per-group K pool is released first
     dims_s = gqla.make_dims(dataclasses.replace(d, k_shared_rope=True))
-    kp_s = torch.empty(tuple(ks[:2]) + (d.G * d.d_nope + d.d_rope,), dtype=d.torch_dtype, device=dev)
+    del graph
+    graph = None
+    kp_shape = tuple(ks[:2]) + (d.G * d.d_nope + d.d_rope,)
+    del kp
+    torch.cuda.empty_cache()
+    kp_s = torch.empty(kp_shape, dtype=d.torch_dtype, device=dev)
     gqla.gqla_expand_cache(dims_s, lay, inp.latent, inp.W_uk, inp.W_uv, kp_s, vp, 0, status)
-    ms_gqa_s = timed(lambda: gqla.gqla_decode_gqa(dims_s, lay, inp.q, kp_s, vp, out_g, lse_g, 0, ws_g, status),
+    ms_gqa_s = timed(lambda: gqla.gqla_decode_gqa(dims_s, lay, inp.q, kp_s, vp, out, lse, 0, ws_g, status),
                      reps) / reps
     del kp_s
+    torch.cuda.empty_cache()
+    kp = torch.empty(ks, dtype=d.torch_dtype, device=dev)
+    gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0, status)
 
-    # end to end through the public API with host buffers: the step's new
-    # inputs (queries and the new tokens' latent rows) go host->device, both
-    # paths' outputs come back device->host, inside the timed region
+    # end to end through the public API with host buffers: the step's inputs
+    # (queries and the new tokens' latent rows) go host->device from pinned
+    # memory, and the step's result (out and lse) comes back device->host,
+    # inside the timed region; every C-ABI call is made on every step, then
+    # the host waits for the step
     q_host = inp.q.cpu().pin_memory()
     new_rows_host = new_rows.cpu().pin_memory()
-    out_host = torch.empty((2,) + tuple(out_a.shape), dtype=out_a.dtype).pin_memory()
+    out_host = torch.empty(tuple(out.shape), dtype=out.dtype).pin_memory()
+    lse_host = torch.empty(tuple(lse.shape), dtype=lse.dtype).pin_memory()
 
-    def e2e_body(run_step):
+    def e2e_body():
         inp.q.copy_(q_host, non_blocking=True)
         new_rows.copy_(new_rows_host, non_blocking=True)
-        run_step()
-        out_host[0].copy_(out_a, non_blocking=True)
-        out_host[1].copy_(out_g, non_blocking=True)
-
-    def e2e_body_overlapped():
-        # each path's output goes to the host as soon as that path is done
-        inp.q.copy_(q_host, non_blocking=True)
-        new_rows.copy_(new_rows_host, non_blocking=True)
-        step_overlapped(after_absorb=lambda: out_host[0].copy_(out_a, non_blocking=True),
-                        after_gqa=lambda: out_host[1].copy_(out_g, non_blocking=True))
-
-    absorb_splits[0], gqa_splits[0] = step_splits
-    # the copies and the step's calls recorded once as a CUDA graph (the copies
-    # read and write the pinned host buffers on every replay), then one replay
-    # and a host wait per step
-    e2e_graph = None
-    if graph is not None:
-        torch.cuda.synchronize()
-        e2e_graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(e2e_graph):
-            e2e_body_overlapped()
+        step()
+        out_host.copy_(out, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
 
     def e2e_step():
-        if e2e_graph is not None:
-            e2e_graph.replay()
-        else:
-            e2e_body(step)
-        torch.cuda.current_stream(dev).synchronize()
+        e2e_body()
+        stream.synchronize()
 
     for _ in range(3):
         e2e_step()
     e2e_ms = timed(e2e_step, args.steps) / args.steps
+    # the same, recorded once as a CUDA graph (copies included) and replayed
+    e2e_graph_ms = None
+    if not args.no_graph:
+        torch.cuda.synchronize()
+        e2e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e2e_graph):
+            e2e_body()
+
+        def e2e_graph_step():
+            e2e_graph.replay()
+            stream.synchronize()
+
+        for _ in range(3):
+            e2e_graph_step()
+        e2e_graph_ms = timed(e2e_graph_step, args.steps) / args.steps
+        del e2e_graph
     clk = clocks.stop() if clocks else None
     torch.cuda.synchronize()
     st = int(status.item())
@@ -471,86 +502,79 @@ def run_ours(args):
     alg = algorithmic(wl)
     tokens = B * d.s_q
     # replicas decode world batches per step; tensor-parallel ranks share one
-    value = multi.job_tokens_per_s(tokens, 1, 1 if tp else world, ms_step)
-    # dominant kernel: the slower decode call of the step
-    if ms_gqa >= ms_absorb:
-        name, ms_dom, bytes_dom = "gqla_decode_gqa", ms_gqa, alg["gqa_bytes"]
-        roof = {"bound": "hbm", "achieved": bytes_dom / (ms_dom * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s"}
+    job = 1 if tp else world
+    value = multi.job_tokens_per_s(tokens, 1, job, ms_step)
+    dec_bytes = alg["absorb_bytes"] if path == gqla.GQLA_PATH_ABSORB else alg["gqa_bytes"]
+    dec_flops = alg["absorb_flops"] if path == gqla.GQLA_PATH_ABSORB else alg["gqa_flops"]
+    # dominant call: the step's decode call, timed live in the eager timed region
+    t_roof, bound = roof_time(dec_bytes, dec_flops, hbm, tf_burst)
+    call = "gqla_decode_%s" % path_name
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": dec_bytes / (ms_decode_live * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s"}
     else:
-        name, ms_dom = "gqla_decode_absorb", ms_absorb
-        t_hbm = alg["absorb_bytes"] / (hbm * 1e9)
-        t_tc = alg["absorb_flops"] / (tf_burst * 1e12)
-        if t_hbm >= t_tc:
-            roof = {"bound": "hbm", "achieved": alg["absorb_bytes"] / (ms_dom * 1e-3) / 1e9, "peak": hbm,
-                    "unit": "GB/s"}
-        else:
-            roof = {"bound": "tensor", "achieved": alg["absorb_flops"] / (ms_dom * 1e-3) / 1e12, "peak": tf_burst,
-                    "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": dec_flops / (ms_decode_live * 1e-3) / 1e12, "peak": tf_burst,
+                "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic(name)
-    roof["kernel"] = name
-    roof["peak_source"] = peak_src
+    roof["traffic"] = recorded_traffic(call, config["workload"])
+    roof["kernel"] = call + (" (one call: absorbed-query GEMM, latent decode, split merge, up-projection)"
+                             if path == gqla.GQLA_PATH_ABSORB else " (one call: decode and split merge)")
+    roof["ms_per_launch"] = ms_decode_live
+    roof["algorithmic_bytes"] = dec_bytes
+    roof["algorithmic_flops"] = dec_flops
+    roof["roofline_ms"] = t_roof * 1e3
+    roof["peak_source"] = peak_src + " (MEASURED_PEAKS.json: copy GB/s, cuBLAS bf16 burst TFLOP/s)"
+    # the step's own roofline: everything the step reads, writes and computes
+    step_bytes = alg["append_bytes"] + alg["expand_new_bytes"] + dec_bytes
+    step_flops = alg["expand_new_flops"] + dec_flops
+    t_step_roof, step_bound = roof_time(step_bytes, step_flops, hbm, tf_burst)
 
     def path_entry(ms, nbytes, flops):
-        t_roof = max(nbytes / (hbm * 1e9), flops / (tf_burst * 1e12))
+        t, bnd = roof_time(nbytes, flops, hbm, tf_burst)
         return {"ms": ms, "tokens_per_s": tokens / (ms * 1e-3), "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
-                "tflops": flops / (ms * 1e-3) / 1e12, "roofline_frac": t_roof / (ms * 1e-3),
-                "bound": "hbm" if nbytes / (hbm * 1e9) >= flops / (tf_burst * 1e12) else "tensor"}
+                "tflops": flops / (ms * 1e-3) / 1e12, "roofline_frac": t / (ms * 1e-3), "bound": bnd}
 
-    T = B * wl.seq_len
-    exp_flops = 2 * T * d.r * d.G * (d.d_nope + d.d_v)
-    exp_bytes = 2 * T * (d.r + d.d_rope) + 2 * T * d.G * (d.d_qk + d.d_v)
     h2d = q_host.numel() * q_host.element_size() + new_rows_host.numel() * new_rows_host.element_size()
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = out_host.numel() * out_host.element_size() + lse_host.numel() * lse_host.element_size()
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if tp else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, random-init weights)",
-        "config": {"workload": "%s B%d L%d s_q%d" % (wl.name, B, wl.seq_len, d.s_q), "batch": B,
-                   "seq_len": wl.seq_len, "s_q": d.s_q, "n_h": d.n_h, "G": d.G, "d_nope": d.d_nope,
-                   "d_rope": d.d_rope, "d_v": d.d_v, "r": d.r,
-                   "step": ("append the s_q new tokens (latent rows + their per-group expansion) + absorb "
-                            "decode + GQA decode"),
-                   "launch": ("cuda_graph replay of the step; absorb path on a second stream, overlapped with "
-                              "the tail expansion + GQA path") if graph is not None else "eager, sequential",
-                   "eager_ms_per_step": eager_ms,
-                   "l2": "no flush: inputs larger than L2 (latent %.0f MB, expanded cache %.0f MB)" % (
-                       alg["absorb_bytes"] / 1e6, alg["gqa_bytes"] / 1e6),
-                   "parallelism": ("tp%d over groups (each rank: G/%d groups and their heads; no collective "
-                                   "inside attention)" % (world, world)) if tp else
-                                  "replicas x%d (batch-sharded, no collective)" % world},
+        "config": config,
+        "step": {"path": path_name,
+                 "selector": {"path": "absorb" if sel_path == gqla.GQLA_PATH_ABSORB else "gqa",
+                              "predicted_absorb_ms": sel_absorb_us * 1e-3, "predicted_gqa_ms": sel_gqa_us * 1e-3},
+                 "calls": ["gqla_append_tokens (new latent rows)", "gqla_append_tokens (their expansion)", call],
+                 "launch": "cuda_graph replay of the step" if not args.no_graph else "eager",
+                 "eager_ms_per_step": eager_ms,
+                 "roofline": {"bound": step_bound, "bytes": step_bytes, "flops": step_flops,
+                              "roofline_ms": t_step_roof * 1e3, "frac": t_step_roof / (ms_step * 1e-3)}},
         "roofline": roof,
-        "e2e": {"value": (1 if tp else world) * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
-                "launch": ("one CUDA graph replay (H2D copies, the step's calls, D2H copies) and a host wait per "
-                           "step") if e2e_graph is not None else "eager calls and a host wait per step",
-                "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+        "e2e": {"value": job * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "launch": "every C-ABI call of the step made eagerly each step, then a host wait",
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e_graph": ({"value": job * tokens / (e2e_graph_ms * 1e-3), "unit": "tokens/s",
+                       "launch": "one CUDA graph replay (H2D copies, the step's calls, D2H copies) and a host "
+                                 "wait per step", "ms_per_step": e2e_graph_ms,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h} if e2e_graph_ms else None),
         "gpu_launches": launches,
+        "gpu_launches_per_step": launches / args.steps,
         "clocks": clk,
         "paths": {"absorb": path_entry(ms_absorb, alg["absorb_bytes"], alg["absorb_flops"]),
                   "gqa": path_entry(ms_gqa, alg["gqa_bytes"], alg["gqa_flops"]),
                   "gqa_shared_rope": path_entry(ms_gqa_s, alg["gqa_shared_bytes"], alg["gqa_flops"]),
-                  "expand_tail": {"ms": ms_tail},
                   "append_latent": {"ms": ms_append},
-                  "append_and_expand": {"ms": ms_append_expand},
-                  "expand_full_cache": {"ms": ms_expand_full, "tflops": exp_flops / (ms_expand_full * 1e-3) / 1e12,
-                                        "hbm_gbs": exp_bytes / (ms_expand_full * 1e-3) / 1e9,
-                                        "tc_frac": exp_flops / (ms_expand_full * 1e-3) / (tf_burst * 1e12)}},
+                  "expand_new_tokens": path_entry(ms_expand_new, alg["expand_new_bytes"], alg["expand_new_flops"]),
+                  "expand_full_cache": path_entry(ms_expand_full, alg["expand_full_bytes"],
+                                                  alg["expand_full_flops"])},
         "splits": {"absorb": gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_ABSORB),
-                   "in_overlapped_step": {
-                       "absorb": gqla.gqla_num_splits(dims, lay, absorb_splits[0], gqla.GQLA_PATH_ABSORB),
-                       "gqa": gqla.gqla_num_splits(dims, lay, gqa_splits[0], gqla.GQLA_PATH_GQA)},
-                   "step_tuning_ms": ({"absorb %s, gqa %s" % (k[0] or "plan", k[1] or "plan"): v
-                                       for k, v in tuned.items()} if tuned else None),
                    "gqa": gqla.gqla_num_splits(dims, lay, 0, gqla.GQLA_PATH_GQA)},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        inp_cpu = inp
-        line["cpu_baseline"] = cpu_baseline(inp_cpu)
+        line["cpu_baseline"] = cpu_baseline(inp)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, e2e_graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -754,10 +778,48 @@ def run_sweep(args):
     return 0
 
 
+def run_once(args):
+    """A few calls of one decode path on a small case (for ncu captures)."""
+    import torch
+    from latent_kv_cache_flash_b200 import build, gqla, synth
+    build.build()
+    wl = synth.dsv3(seq_len=args.seq_len, s_q=args.sq, batch=args.batch, G=args.groups)
+    inp = synth.make_inputs(wl, "cuda")
+    d = wl.dims
+    dims = gqla.make_dims(d)
+    lay = gqla.make_layout(inp.seq_lens, inp.max_seq_len, 0, inp.capacity)
+    out = torch.empty((wl.batch, d.s_q, d.n_h, d.d_v), dtype=d.torch_dtype, device="cuda")
+    lse = torch.empty((wl.batch, d.s_q, d.n_h), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if args.once == "absorb":
+        ws = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_ABSORB, "cuda")
+        fn = lambda: gqla.gqla_decode_absorb(dims, lay, inp.q, inp.latent, inp.W_uk, inp.W_uv, out, lse, 0, ws,
+                                             status)
+    else:
+        ks, vs = synth.expanded_pool_shapes(inp)
+        kp = torch.empty(ks, dtype=d.torch_dtype, device="cuda")
+        vp = torch.empty(vs, dtype=d.torch_dtype, device="cuda")
+        gqla.gqla_expand_cache(dims, lay, inp.latent, inp.W_uk, inp.W_uv, kp, vp, 0, status)
+        ws = gqla.workspace_for(dims, lay, 0, gqla.GQLA_PATH_GQA, "cuda")
+        fn = lambda: gqla.gqla_decode_gqa(dims, lay, inp.q, kp, vp, out, lse, 0, ws, status)
+    for _ in range(args.warmup + 1):
+        fn()
+    torch.cuda.synchronize()
+    st = int(status.item())
+    path = gqla.GQLA_PATH_ABSORB if args.once == "absorb" else gqla.GQLA_PATH_GQA
+    print(json.dumps({"once": args.once, "workload": "%s B%d L%d G%d s_q%d" % (wl.name, wl.batch, wl.seq_len, d.G,
+                                                                                  d.s_q),
+                      "splits": gqla.gqla_num_splits(dims, lay, 0, path), "calls": args.warmup + 1,
+                      "status": st}))
+    return 0 if st == 0 else 1
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.once:
+        return run_once(args)
     if args.sweep:
         return run_sweep(args)
     return run_ours(args)

@@ -18,8 +18,10 @@
  * Conventions shared by every entry point:
  *  - All pointers named *device* are CUDA device pointers owned by the caller;
  *    the library never allocates device memory (split-KV scratch is passed in
- *    as a workspace) and never frees anything.  Host structs are read during
- *    the call only.
+ *    as a workspace) and never frees anything.  The one exception is
+ *    gqla_decode_gqa_noalloc, whose split scratch is a fixed 32 MiB
+ *    library-owned __device__ array (described at that call).  Host structs
+ *    are read during the call only.
  *  - Work is queued on `stream` (a cudaStream_t; NULL = legacy default stream)
  *    and runs asynchronously; no call synchronises.
  *  - Arguments are validated on the host before any launch; a failed check
@@ -217,6 +219,9 @@ gqla_status gqla_decode_gqa(const gqla_dims* dims, const gqla_kv_layout* layout,
  *   GQLA_ERR_WORKSPACE before any launch: pass a smaller num_splits.
  *   The first call on each device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
+ *   The address is kept with the CUDA context it belongs to: after a device
+ *   reset, or when that context is replaced, the next call looks it up again
+ *   (so that call, too, belongs outside a stream capture).
  *   All calls share the one array, so calls whose kernels may overlap on the
  *   GPU (different streams, or other threads) race: serialise them. */
 gqla_status gqla_decode_gqa_noalloc(const gqla_dims* dims, const gqla_kv_layout* layout,

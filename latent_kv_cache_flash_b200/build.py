@@ -78,7 +78,7 @@ def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False)
         any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs)
     if relink:
         tmp = LIB + ".tmp"
-        cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcuda"]
+        cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)

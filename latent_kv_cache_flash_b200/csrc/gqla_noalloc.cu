@@ -4,6 +4,8 @@
 // needs no allocation at all: for hosts that own every byte of device memory
 // and hand a plug-in none of it, and for decode loops that may not call an
 // allocator on the hot path (cudaMalloc/cudaFree synchronise the device).
+#include <cuda.h>
+
 #include <mutex>
 
 #include "gqla.h"
@@ -20,28 +22,60 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 // Device address of the scratch array for the current device.  In host code
 // g_noalloc_scratch names a host-side stand-in, not device memory, so the
-// address is looked up once per device (with that device current) and cached.
+// address is looked up with that device current.  It is cached per device
+// together with the context it was looked up in: a device reset or a new
+// primary context loads the module afresh, so a changed context triggers a
+// new lookup instead of reusing a stale address.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, looked up once through the runtime (the
+// library does not link libcuda).
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (CtxGetCurrentFn)f;
+  }
+  return fn;
+}
+
+CUcontext current_context() {
+  CtxGetCurrentFn fn = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
 void* scratch_for_current_device(gqla_status* status) {
   static std::mutex mu;
   static void* cached[64] = {nullptr};
+  static CUcontext cached_ctx[64] = {nullptr};
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     *status = GQLA_ERR_CUDA;
     return nullptr;
   }
+  // the context current on this thread (none before the runtime's first call
+  // here; the symbol lookup below creates the device's primary context then)
+  CUcontext ctx = current_context();
   std::lock_guard<std::mutex> lock(mu);
-  if (!cached[dev]) {
-    void* ptr = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || ptr == nullptr) {
-      cudaGetLastError();
-      *status = GQLA_ERR_CUDA;
-      return nullptr;
-    }
-    cached[dev] = ptr;
+  if (ctx != nullptr && cached[dev] != nullptr && cached_ctx[dev] == ctx) return cached[dev];
+  void* ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e == cudaSuccess) ctx = current_context();
+  if (e != cudaSuccess || ptr == nullptr || ctx == nullptr) {
+    cudaGetLastError();
+    cached[dev] = nullptr;
+    *status = GQLA_ERR_CUDA;
+    return nullptr;
   }
-  return cached[dev];
+  cached[dev] = ptr;
+  cached_ctx[dev] = ctx;
+  return ptr;
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }

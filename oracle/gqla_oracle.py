@@ -26,7 +26,7 @@ Sources (web pages on Group-Query Latent Attention):
   GQLAAttention docstring: knob names (decode_path, num_groups), the
   divisibility rule, causal masking in decoder mode.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 head h belongs to group g = h // m with m = n_h / G; the key of token t for
 group g is [c_t W_uk^g ; k_rope_t] (the decoupled RoPE key is shared by all
 heads and already rotated); the value is c_t W_uv^g; the cache of length L

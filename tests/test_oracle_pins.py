@@ -297,3 +297,57 @@ def test_planted_group_map_mistake_caught_by_sdpa():
     right = O.decode_sequence_gqa(q[0], c[0], kr[0], W_uk, W_uv, L, 0.3)[0]
     np.testing.assert_allclose(right, ref, rtol=1e-11, atol=1e-12)
     assert m == 4
+
+
+# --- the batch driver -------------------------------------------------------
+
+def _ragged_batch(seed, lens, s_q=2):
+    """Three sequences of different lengths, each with its own rows; the
+    logical rows past a sequence's length are never read."""
+    rng = np.random.default_rng(seed)
+    n_h, G, d_n, d_r, d_v, r = 4, 2, 3, 2, 3, 5
+    q = rng.standard_normal((len(lens), s_q, n_h, d_n + d_r))
+    c_list = [rng.standard_normal((L + 3, r)) for L in lens]
+    kr_list = [rng.standard_normal((L + 3, d_r)) for L in lens]
+    W_uk = rng.standard_normal((G, r, d_n)) / math.sqrt(r)
+    W_uv = rng.standard_normal((G, r, d_v)) / math.sqrt(r)
+    return q, c_list, kr_list, W_uk, W_uv
+
+
+@pytest.mark.parametrize("form", ["gqa", "absorb"])
+def test_decode_batch_ragged_brute_force(form):
+    """decode_batch over a ragged batch (lengths 2, 7, 4; s_q 2) equals the
+    definition written out for every sequence with its own length and rows."""
+    lens = [2, 7, 4]
+    q, c_list, kr_list, W_uk, W_uv = _ragged_batch(31, lens)
+    o, l = O.decode_batch(q, c_list, kr_list, W_uk, W_uv, np.array(lens), 0.41, form=form)
+    assert o.shape == (3, 2, 4, 3) and l.shape == (3, 2, 4)
+    for b, L in enumerate(lens):
+        bo, bl = _brute_force(q[b], c_list[b], kr_list[b], W_uk, W_uv, L, 0.41)
+        np.testing.assert_allclose(o[b], bo, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(l[b], bl, rtol=1e-12, atol=1e-13)
+
+
+def test_decode_batch_planted_mistakes_caught(monkeypatch):
+    """A batch driver that decodes every sequence with the first one's length,
+    or reads the next sequence's rows, fails the brute-force pin above."""
+    lens = [2, 7, 4]
+    q, c_list, kr_list, W_uk, W_uv = _ragged_batch(31, lens)
+
+    def pinned(res):
+        o, l = res
+        for b, L in enumerate(lens):
+            bo, bl = _brute_force(q[b], c_list[b], kr_list[b], W_uk, W_uv, L, 0.41)
+            if not (np.allclose(o[b], bo, rtol=1e-12, atol=1e-13) and np.allclose(l[b], bl, rtol=1e-12, atol=1e-13)):
+                return False
+        return True
+
+    assert pinned(O.decode_batch(q, c_list, kr_list, W_uk, W_uv, np.array(lens), 0.41))
+    first_len = np.array([lens[0]] * 3)
+    assert not pinned(O.decode_batch(q, c_list, kr_list, W_uk, W_uv, first_len, 0.41))
+    shifted = c_list[1:] + c_list[:1]
+    shifted_kr = kr_list[1:] + kr_list[:1]
+    # rows of sequence b + 1 with the right lengths (trimmed to fit the shorter buffers)
+    rows = [np.resize(shifted[b], c_list[b].shape) for b in range(3)]
+    rows_kr = [np.resize(shifted_kr[b], kr_list[b].shape) for b in range(3)]
+    assert not pinned(O.decode_batch(q, rows, rows_kr, W_uk, W_uv, np.array(lens), 0.41))
