@@ -58,7 +58,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="dsv3_64k", choices=WORKLOADS)
-    ap.add_argument("--sq", type=int, default=1, choices=[1, 2])
+    ap.add_argument("--sq", type=int, default=1, choices=[1, 2, 3, 4])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", choices=["select", "absorb", "gqa"], default="select",
                     help="decode path of the step: the library's selector (default) or a fixed one")

@@ -25,6 +25,20 @@ def tol(dtype: str, ref: np.ndarray) -> float:
 # log-sum-exp error (lse grows like ln L) are the sharper readings.
 DIAG = []
 
+# Sharper gates at long context (bf16, every sampled sequence >= 8192 tokens).
+# The lse is compared in absolute terms: it grows like ln L while its error
+# shrinks as the per-score rounding errors (q~ or the expanded K rounded to
+# bf16, about 2^-9 relative per product, independent across tokens) average
+# out over the softmax weights; measured at most 3.2e-4 at 8K-64K on B200, so
+# 2e-3 keeps a margin of six and is 55 times tighter than the output rule
+# gives it at L = 64K (1e-2 * 11.7 + 1e-3).  The output's relative RMS error
+# is bounded by the few bf16 roundings on the way (P, the merged latent
+# output, the expanded cache: each about 2^-9 / sqrt(3) = 1.1e-3 relative RMS),
+# measured at most 3.0e-3; the gate is 1e-2.
+LONG_CONTEXT = 8192
+LSE_ABS_TOL_LONG = 2e-3
+OUT_REL_RMS_TOL_LONG = 1e-2
+
 
 def rel_rms(got, ref):
     den = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
@@ -115,8 +129,17 @@ def check_units(inp: synth.Inputs, out, lse, units, what=""):
         got_l.append(l_np[b, :, hs])
         ref_o.append(ref[b][0][:, hs])
         ref_l.append(ref[b][1][:, hs])
-    e1 = assert_close(np.stack(got_o), np.stack(ref_o), d.dtype, what + " out", record=True)
-    e2 = assert_close(np.stack(got_l), np.stack(ref_l), d.dtype, what + " lse", record=True)
+    go, ro, gl, rl = np.stack(got_o), np.stack(ref_o), np.stack(got_l), np.stack(ref_l)
+    e1 = assert_close(go, ro, d.dtype, what + " out", record=True)
+    e2 = assert_close(gl, rl, d.dtype, what + " lse", record=True)
+    if d.dtype == "bf16" and min(inp.seq_lens_host[b] for b, _ in units) >= LONG_CONTEXT:
+        fin = np.isfinite(rl)
+        dl = float(np.max(np.abs(gl[fin].astype(np.float64) - rl[fin]))) if fin.any() else 0.0
+        assert dl <= LSE_ABS_TOL_LONG, "%s: max|d lse| %.3e > %.1e at L >= %d" % (what, dl, LSE_ABS_TOL_LONG,
+                                                                                 LONG_CONTEXT)
+        rr = rel_rms(go.astype(np.float64)[np.isfinite(ro)], ro[np.isfinite(ro)])
+        assert rr <= OUT_REL_RMS_TOL_LONG, "%s: out rel-RMS %.2e > %.1e at L >= %d" % (
+            what, rr, OUT_REL_RMS_TOL_LONG, LONG_CONTEXT)
     return e1, e2
 
 
