@@ -81,16 +81,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
+  // the row blocks of one (sequence, group, split) are neighbours in the grid,
+  // so they run together and read each K/V tile from HBM once, through L2
+  const int split = blockIdx.x / p.rblocks, rb = blockIdx.x % p.rblocks;
   const int b = blockIdx.y / p.G, g = blockIdx.y % p.G;
-  const int rb = blockIdx.z;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&q_full, 4);
     ptx::mbar_init(&qk_drain, 1);
     ptx::mbar_init(&pv_drain, 1);
     for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(&kv_full[s], 1);
+      ptx::mbar_init(&kv_full[s], 2);
       ptx::mbar_init(&kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -115,8 +116,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t_stop = L < 0 ? t_begin : min(t_begin + p.plan.chunk, L);
   const int n_tiles = t_stop > t_begin ? (t_stop - t_begin + kT - 1) / kT : 0;
 
-  if (warp == 0) {
-    // ------------------------------------------------------- TMA producer
+  if (warp == 0 || warp == 7) {
+    // ---------------------------------------------------- TMA producers
+    // One issuing thread brings about 27 bytes per cycle into an SM; the
+    // tile needs more at the tensor pipe's pace, so warp 0 loads the K
+    // chunks and warp 7 the V chunks, both arriving on the stage's barrier.
+    const bool kside = warp == 0;
     if (lane == 0 && n_tiles > 0) {
       ptx::prefetch_tmap(&kmap);
       ptx::prefetch_tmap(&vmap);
@@ -131,12 +136,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*(volatile int*)&abort_flag) break;
         const int row0 = (int)token_row(p.ly, b, t_begin + j * kT, nullptr);
         uint8_t* dst = sKV + s * kStageBytes;
-        ptx::mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
-        ptx::tma_load_2d(dst, &kmap, &kv_full[s], p.kr.nope_at(g), row0);
-        ptx::tma_load_2d(dst + kChunkBytes, &kmap, &kv_full[s], p.kr.nope_at(g) + 64, row0);
-        ptx::tma_load_2d(dst + 2 * kChunkBytes, &kmap, &kv_full[s], p.kr.rope_at(g), row0);
-        for (int c = 0; c < kVChunks; ++c)
-          ptx::tma_load_2d(dst + (kKChunks + c) * kChunkBytes, &vmap, &kv_full[s], g * kDv + 64 * c, row0);
+        if (kside) {
+          ptx::mbar_arrive_expect_tx(&kv_full[s], kKChunks * kChunkBytes);
+          ptx::tma_load_2d(dst, &kmap, &kv_full[s], p.kr.nope_at(g), row0);
+          ptx::tma_load_2d(dst + kChunkBytes, &kmap, &kv_full[s], p.kr.nope_at(g) + 64, row0);
+          ptx::tma_load_2d(dst + 2 * kChunkBytes, &kmap, &kv_full[s], p.kr.rope_at(g), row0);
+        } else {
+          ptx::mbar_arrive_expect_tx(&kv_full[s], kVChunks * kChunkBytes);
+          for (int c = 0; c < kVChunks; ++c)
+            ptx::tma_load_2d(dst + (kKChunks + c) * kChunkBytes, &vmap, &kv_full[s], g * kDv + 64 * c, row0);
+        }
         issued = j + 1;
       }
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
@@ -463,7 +472,7 @@ cudaError_t tc_gqa_wide_decode(const Problem& p, const void* q, const void* k_po
   prm.kr = p.kr;
   cudaError_t e = ensure_smem_limit((const void*)gqa_wide_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.plan.num_splits, p.ly.batch * d.G, prm.rblocks);
+  dim3 grid(p.plan.num_splits * prm.rblocks, p.ly.batch * d.G);
   gqa_wide_kernel<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, prm);
   count_launch();
   return cudaGetLastError();
