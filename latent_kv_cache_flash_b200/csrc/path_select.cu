@@ -19,14 +19,23 @@ namespace {
 constexpr double kDefaultHbmGbs = 6559.0;
 constexpr double kDefaultTcTflops = 1656.2;
 
-// Efficiencies of the kernels against those two rates (measured over the
-// crossover grid n_h 128, G 1..128, s_q 1..4, B32, L 32K):
-constexpr double kEtaStream = 1.08;     // GQA mma.sync kernel: K/V read stream (1.07..1.10 of the copy rate at G >= 8)
-constexpr double kEtaWideTc = 0.40;     // GQA tcgen05 kernel: softmax-bound 128-row tiles (two warpgroups)
+// Efficiencies of the kernels against those two rates, and their fixed
+// costs, measured on a B200 over the crossover grid (n_h 128, G 1..128,
+// s_q 1..4, B32, L 32K) and the DeepSeek-V3-shaped context sweep (B64,
+// L 8K..64K):
+constexpr double kEtaStream = 1.08;     // GQA mma.sync kernel, <= 16 rows a group: K/V read stream (1.07..1.10 of the copy rate)
+constexpr double kEtaStreamWide = 1.0;  // the same kernel at 17..63 rows a group, where its MMAs slow each CTA's stream
+constexpr double kEtaWideTc = 0.54;     // GQA tcgen05 kernel: a 128-row block-tile, full or not (softmax-bound)
+constexpr double kEtaWideBw = 0.94;     // its K/V stream, paid by the first row block of a tile (the others hit L2)
+constexpr double kWideCtaUs = 11.0;     // its CTA prologue (query into TMEM) + epilogue (merge of two states, output)
 constexpr double kEtaAbsorbTc = 0.41;   // absorb tcgen05 kernel: M=64 tiles, N=64 score MMAs
 constexpr double kEtaAbsorbBw = 0.90;   // absorb latent stream when the tensor side keeps up
 constexpr double kLaunchUs = 3.0;       // one kernel launch on a busy stream
 constexpr double kAbsorbCtaUs = 8.0;    // absorb CTA prologue (q~ into TMEM) + epilogue (64 x 512 fp32 out)
+// The absorbed-query GEMM and the up-projection are latency-bound small
+// GEMMs: 18 and 26 us at 8192 rows, 9 and 7.5 us at 1024 rows.
+constexpr double kAbsorbQUs = 7.7, kAbsorbQUsPerRow = 1.26e-3;
+constexpr double kUpProjUs = 7.5, kUpProjUsPerRow = 2.3e-3;
 
 struct Rates {
   double bw_sm;   // bytes/us per SM
@@ -35,10 +44,9 @@ struct Rates {
   int sms;
 };
 
-// Split partials written by the decode kernel and read by the combine.
+// Split partials read back by the merge (their writes overlap the decode).
 double combine_us(const Problem& p, int D, const Rates& r) {
-  if (p.plan.num_splits <= 1) return 0.0;
-  const double bytes = 2.0 * p.plan.num_splits * (double)p.rows * (D + 1) * 4;
+  const double bytes = (double)p.plan.num_splits * (double)p.rows * (D + 1) * 4;
   return bytes / r.bw + kLaunchUs;
 }
 
@@ -50,11 +58,12 @@ double absorb_us(const Problem& p, long long T, const Rates& r) {
   const double flops_tile = 2.0 * 64 * 64 * (2.0 * d.r + d.d_rope);   // QK over r + d_rope, PV over r
   const double bytes_tile = 64.0 * (d.r + d.d_rope) * es;
   const double t_tile = fmax(flops_tile / (r.tc_sm * kEtaAbsorbTc), bytes_tile / (r.bw_sm * kEtaAbsorbBw));
+  // one CTA per SM: whole waves of CTAs, each its share of the tiles
   const double ctas = (double)p.ly.batch * p.plan.num_splits * rb;
-  const double busy = fmin(ctas, (double)r.sms);
-  const double dec = ceil(ctas / r.sms) * kAbsorbCtaUs + tiles * rb * t_tile / busy;
-  // absorbed-query GEMM + latent combine + up-projection
-  const double aux = 3 * kLaunchUs + combine_us(p, d.r, r);
+  const double dec = ceil(ctas / r.sms) * (kAbsorbCtaUs + tiles * rb / ctas * t_tile);
+  // absorbed-query GEMM + merge of the split partials + up-projection
+  const double aux = kAbsorbQUs + kAbsorbQUsPerRow * p.rows + combine_us(p, d.r, r) + kUpProjUs +
+                     kUpProjUsPerRow * p.rows;
   return dec + aux;
 }
 
@@ -67,13 +76,14 @@ double gqa_us(const Problem& p, long long T, const Rates& r) {
   if (tc_gqa_wide_supports(p)) {
     const long long rb = (p.m * d.s_q + 127) / 128;
     const double flops_tile = 2.0 * 128 * 64 * (p.d_qk + d.d_v);
-    const double bytes_tile = 64.0 * row_bytes / d.G;
-    const double t_tile = fmax(flops_tile / (r.tc_sm * kEtaWideTc), bytes_tile / (r.bw_sm * kEtaStream));
-    dec = tiles * d.G * rb * t_tile / r.sms;
+    const double bytes_tile = 64.0 * row_bytes / d.G / rb;
+    const double t_tile = fmax(flops_tile / (r.tc_sm * kEtaWideTc), bytes_tile / (r.bw_sm * kEtaWideBw));
+    const double ctas = (double)p.ly.batch * d.G * p.plan.num_splits * rb;
+    dec = ceil(ctas / r.sms) * (kWideCtaUs + tiles * d.G * rb / ctas * t_tile);
   } else {
-    dec = (double)T * row_bytes / (r.bw * kEtaStream);
+    dec = (double)T * row_bytes / (r.bw * (p.m * d.s_q <= 16 ? kEtaStream : kEtaStreamWide));
   }
-  return dec + kLaunchUs + combine_us(p, d.d_v, r);
+  return dec + kLaunchUs + (p.plan.num_splits > 1 ? combine_us(p, d.d_v, r) : 0.0);
 }
 
 }  // namespace

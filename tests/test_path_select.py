@@ -15,13 +15,22 @@ B200 = (148, 6559.0, 1656.2)   # SMs, copy GB/s, dense bf16 TFLOP/s (measured on
 # d = v = 128, B32, L 32K), measured on one B200 with `bench.py --sweep
 # crossover` (absorb ms, GQA ms).  A performance record, not an oracle value.
 MEASURED_B200 = {
-    (1, 1): (0.506, 0.151), (1, 2): (0.954, 0.286), (1, 4): (1.768, 0.535),
-    (2, 1): (0.505, 0.275), (2, 2): (0.955, 0.281), (2, 4): (1.770, 0.536),
-    (4, 1): (0.504, 0.489), (4, 2): (0.955, 0.514), (4, 4): (1.770, 0.537),
-    (8, 1): (0.510, 0.759), (8, 2): (0.989, 0.861), (8, 4): (1.841, 0.961),
-    (16, 1): (0.539, 1.512), (16, 2): (0.958, 1.512), (16, 4): (1.800, 1.627),
-    (32, 1): (0.508, 2.987), (32, 2): (0.958, 3.002), (32, 4): (1.776, 3.033),
-    (128, 1): (0.509, 12.192), (128, 2): (0.963, 12.198), (128, 4): (1.777, 12.210),
+    (1, 1): (0.508, 0.153), (1, 2): (0.954, 0.256), (1, 4): (1.767, 0.463),
+    (2, 1): (0.506, 0.277), (2, 2): (0.953, 0.284), (2, 4): (1.768, 0.480),
+    (4, 1): (0.504, 0.485), (4, 2): (0.955, 0.516), (4, 4): (1.767, 0.538),
+    (8, 1): (0.506, 0.760), (8, 2): (0.954, 0.856), (8, 4): (1.769, 0.967),
+    (16, 1): (0.521, 1.513), (16, 2): (0.960, 1.512), (16, 4): (1.771, 1.624),
+    (32, 1): (0.513, 2.984), (32, 2): (0.981, 3.000), (32, 4): (1.771, 3.029),
+    (128, 1): (0.509, 12.188), (128, 2): (0.961, 12.174), (128, 4): (1.773, 12.187),
+}
+
+# The DeepSeek-V3-shaped layer (n_h 128, G 16, B64) over context lengths,
+# `bench.py --sweep context` on the same B200: (L, s_q) -> (absorb ms, GQA ms).
+MEASURED_CONTEXT_B200 = {
+    (8192, 1): (0.310, 0.778), (8192, 2): (0.582, 0.804),
+    (16384, 1): (0.534, 1.507), (16384, 2): (1.014, 1.531),
+    (32768, 1): (0.972, 2.979), (32768, 2): (1.795, 3.003),
+    (65536, 1): (1.761, 5.970), (65536, 2): (3.354, 6.006),
 }
 
 
@@ -44,9 +53,17 @@ def test_reproduces_the_measured_crossover(G):
         path, a_us, g_us = _est(G, 128, groups, s_q, 32, 32768)
         want = G.GQLA_PATH_GQA if ms_g < ms_a else G.GQLA_PATH_ABSORB
         assert path == want, (groups, s_q, a_us, g_us)
-        # and the predicted times are within 25% of the measured ones
-        assert abs(a_us / (ms_a * 1e3) - 1) < 0.25, (groups, s_q, a_us, ms_a)
-        assert abs(g_us / (ms_g * 1e3) - 1) < 0.25, (groups, s_q, g_us, ms_g)
+        # and the predicted times are within 15% of the measured ones
+        assert abs(a_us / (ms_a * 1e3) - 1) < 0.15, (groups, s_q, a_us, ms_a)
+        assert abs(g_us / (ms_g * 1e3) - 1) < 0.15, (groups, s_q, g_us, ms_g)
+
+
+def test_reproduces_the_measured_context_sweep(G):
+    for (L, s_q), (ms_a, ms_g) in MEASURED_CONTEXT_B200.items():
+        path, a_us, g_us = _est(G, 128, 16, s_q, 64, L)
+        assert path == (G.GQLA_PATH_GQA if ms_g < ms_a else G.GQLA_PATH_ABSORB), (L, s_q)
+        assert abs(a_us / (ms_a * 1e3) - 1) < 0.10, (L, s_q, a_us, ms_a)
+        assert abs(g_us / (ms_g * 1e3) - 1) < 0.10, (L, s_q, g_us, ms_g)
 
 
 def test_structure_of_the_estimates(G):
@@ -58,10 +75,12 @@ def test_structure_of_the_estimates(G):
         assert abs(t1 / t0 - g1 / g0) < 0.02 * g1 / g0
     # the shared-RoPE K pool streams fewer bytes
     assert _est(G, 128, 16, 1, 64, 16384, shared=True)[2] < _est(G, 128, 16, 1, 64, 16384)[2]
-    # doubling the context doubles both (long-context regime)
+    # doubling the context nearly doubles both (long-context regime); the
+    # absorbed call's side GEMMs and merge do not grow with L (measured: 0.534
+    # -> 0.972 ms, a factor 1.82)
     p1, a1, g1 = _est(G, 128, 16, 1, 64, 16384)
     p2, a2, g2 = _est(G, 128, 16, 1, 64, 32768)
-    assert 1.8 < a2 / a1 < 2.1 and 1.9 < g2 / g1 < 2.1
+    assert 1.7 < a2 / a1 < 2.1 and 1.9 < g2 / g1 < 2.1
 
 
 def test_preference_follows_the_compute_to_bandwidth_ratio(G):
