@@ -28,14 +28,14 @@ constexpr double kEtaStreamWide = 1.0;  // the same kernel at 17..63 rows a grou
 constexpr double kEtaWideTc = 0.54;     // GQA tcgen05 kernel: a 128-row block-tile, full or not (softmax-bound)
 constexpr double kEtaWideBw = 0.94;     // its K/V stream, paid by the first row block of a tile (the others hit L2)
 constexpr double kWideCtaUs = 11.0;     // its CTA prologue (query into TMEM) + epilogue (merge of two states, output)
-constexpr double kEtaAbsorbTc = 0.41;   // absorb tcgen05 kernel: M=64 tiles, N=64 score MMAs
-constexpr double kEtaAbsorbBw = 0.90;   // absorb latent stream when the tensor side keeps up
+constexpr double kEtaAbsorbTc = 0.42;   // absorb tcgen05 kernel: M=64 tiles, N=64 score MMAs
+constexpr double kEtaAbsorbBw = 0.90;   // a CTA's latent tile loads (every row block loads each tile into its SM)
 constexpr double kLaunchUs = 3.0;       // one kernel launch on a busy stream
-constexpr double kAbsorbCtaUs = 8.0;    // absorb CTA prologue (q~ into TMEM) + epilogue (64 x 512 fp32 out)
-// The absorbed-query GEMM and the up-projection are latency-bound small
-// GEMMs: 18 and 26 us at 8192 rows, 9 and 7.5 us at 1024 rows.
-constexpr double kAbsorbQUs = 7.7, kAbsorbQUsPerRow = 1.26e-3;
-constexpr double kUpProjUs = 7.5, kUpProjUsPerRow = 2.3e-3;
+constexpr double kAbsorbCtaUs = 9.0;    // absorb CTA prologue (q~ into TMEM) + epilogue (64 x 512 fp32 out)
+// The absorbed-query GEMM and the fused split merge + up-projection, beside
+// reading the split partials back: latency-bound small launches, about 31 us
+// together from 4K to 16K rows.
+constexpr double kAbsorbSideUs = 31.0;
 
 struct Rates {
   double bw_sm;   // bytes/us per SM
@@ -61,9 +61,8 @@ double absorb_us(const Problem& p, long long T, const Rates& r) {
   // one CTA per SM: whole waves of CTAs, each its share of the tiles
   const double ctas = (double)p.ly.batch * p.plan.num_splits * rb;
   const double dec = ceil(ctas / r.sms) * (kAbsorbCtaUs + tiles * rb / ctas * t_tile);
-  // absorbed-query GEMM + merge of the split partials + up-projection
-  const double aux = kAbsorbQUs + kAbsorbQUsPerRow * p.rows + combine_us(p, d.r, r) + kUpProjUs +
-                     kUpProjUsPerRow * p.rows;
+  // absorbed-query GEMM + merge of the split partials and up-projection
+  const double aux = kAbsorbSideUs + (double)p.plan.num_splits * (double)p.rows * (d.r + 1) * 4 / r.bw;
   return dec + aux;
 }
 

@@ -44,9 +44,9 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
 bool gemm_absorb_q_supports(const Problem& p);
 cudaError_t absorb_q_mma(const Problem& p, const void* q, const void* W_uk, __nv_bfloat16* qt, cudaStream_t s);
 bool gemm_combine_up_supports(const Problem& p);
-// o_lat: bf16 [rows, r] scratch for the merged latent output.
+// The split merge of the latent output and the up-projection, one launch.
 cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const float* lse_part, const void* W_uv,
-                           void* out, float* lse_out, __nv_bfloat16* o_lat, cudaStream_t s);
+                           void* out, float* lse_out, cudaStream_t s);
 
 // Cache expansion GEMM on tcgen05 (tc_expand.cu).
 bool tc_expand_supports(const Problem& p);

@@ -453,7 +453,7 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (gemm_combine_up_supports(p))
-    return combine_up_mma(p, S, w.o_part, w.lse_part, W_uv, out, lse, (__nv_bfloat16*)w.o_lat, s);
+    return combine_up_mma(p, S, w.o_part, w.lse_part, W_uv, out, lse, s);
   e = combine(S, p.rows, kR, w.o_part, w.lse_part, w.o_lat, GQLA_F32, lse, s);
   if (e != cudaSuccess) return e;
   return simt_up_proj(p, w.o_lat, W_uv, out, s);

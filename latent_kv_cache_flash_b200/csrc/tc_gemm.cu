@@ -1,10 +1,12 @@
 // Small bf16 GEMMs around the decode kernels, on mma.sync m16n8k16 tiles
 // (fp32 accumulate):
-//  * absorb_q:      q~[row] = W_uk^g q_nope[row]          (per group, r outputs)
-//  * combine_lat + up_proj: LSE merge of the split partials of the latent
-//                   output (bf16), then out[row] = o_lat[row] W_uv^g
+//  * absorb_q:  q~[row] = W_uk^g q_nope[row]              (per group, r outputs)
+//  * merge_up:  LSE merge of the split partials of the latent output (rounded
+//               to bf16 in shared memory), then out[row] = o_lat[row] W_uv^g,
+//               in one launch
 // They read their row-major operands through ldmatrix from padded shared
-// memory; the weight operand is shared by every row of a group.
+// memory; the weight operand is shared by every row of a group, so a CTA
+// takes 64 rows of one group to load each weight slice once per 64 rows.
 #include <math.h>
 
 #include "ptx.cuh"
@@ -15,6 +17,15 @@ namespace gqla {
 namespace {
 
 using bf16 = __nv_bfloat16;
+
+// 16-byte global -> shared copies that do not hold the issuing thread; a
+// false predicate fills the destination with zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool pred) {
+  const int sz = pred ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void ldsm_a(uint32_t base, int pitch_bytes, int row0, int k0, uint32_t* a) {
   const int lane = threadIdx.x & 31;
@@ -38,11 +49,12 @@ __device__ __forceinline__ void ldsm_b_kn(uint32_t base, int pitch_bytes, int n0
 }
 
 // ------------------------------------------------------------- absorb_q
-// CTA: 32 rows of group g x 128 outputs; 4 warps = 2 row blocks x 2 output
-// halves.  K = d_nope.
-constexpr int kAqRows = 32, kAqN = 128, kAqMaxK = 256;
+// CTA: 64 rows of group g x 128 outputs; 8 warps = 4 row blocks x 2 output
+// halves.  K = d_nope.  Both operands come in through cp.async, all in
+// flight at once.
+constexpr int kAqRows = 64, kAqN = 128, kAqMaxK = 256, kAqThreads = 256;
 
-__global__ void __launch_bounds__(128) absorb_q_mma_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_uk,
+__global__ void __launch_bounds__(kAqThreads) absorb_q_mma_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_uk,
                                                            bf16* __restrict__ qt, int rows_g, int n_h, int m,
                                                            int d_n, int d_qk, int r) {
   extern __shared__ __align__(16) uint8_t sm[];
@@ -51,28 +63,25 @@ __global__ void __launch_bounds__(128) absorb_q_mma_kernel(const bf16* __restric
   uint8_t* sA = sm;
   uint8_t* sB = sm + kAqRows * pitch;
   const int gran = d_n / 8;
+  const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
   for (int i = threadIdx.x; i < kAqRows * gran; i += blockDim.x) {
     const int rr = i / gran, c = i % gran;
     const int lr = blockIdx.x * kAqRows + rr;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (lr < rows_g) {
-      const long long grow = (long long)(lr / m) * n_h + g * m + lr % m;
-      v = *reinterpret_cast<const uint4*>(q + grow * d_qk + c * 8);
-    }
-    *reinterpret_cast<uint4*>(sA + rr * pitch + c * 16) = v;
+    const long long grow = lr < rows_g ? (long long)(lr / m) * n_h + g * m + lr % m : 0;
+    cp_async16(a_base + rr * pitch + c * 16, q + grow * d_qk + c * 8, lr < rows_g);
   }
   for (int i = threadIdx.x; i < kAqN * gran; i += blockDim.x) {
     const int nn = i / gran, c = i % gran;
-    *reinterpret_cast<uint4*>(sB + nn * pitch + c * 16) =
-        *reinterpret_cast<const uint4*>(W_uk + ((size_t)g * r + n0 + nn) * d_n + c * 8);
+    cp_async16(b_base + nn * pitch + c * 16, W_uk + ((size_t)g * r + n0 + nn) * d_n + c * 8, true);
   }
+  cp_async_commit();
+  cp_async_wait0();
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wr = warp & 1, wn = warp >> 1;
+  const int wr = warp & 3, wn = warp >> 2;
   float acc[kAqN / 16][4];
 #pragma unroll
   for (int n = 0; n < kAqN / 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-  const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
   for (int k0 = 0; k0 < d_n; k0 += 16) {
     uint32_t a[4];
     ldsm_a(a_base, pitch, wr * 16, k0, a);
@@ -97,86 +106,28 @@ __global__ void __launch_bounds__(128) absorb_q_mma_kernel(const bf16* __restric
   }
 }
 
-// --------------------------------------------------------- combine_lat
-// LSE merge of the split partials of the absorb path's latent output, one
-// warp per (row, 128-column quarter); output rounded to bf16 for the
-// up-projection's A operand.
+// ------------------------------------------------------------ merge_up
+// out[row] = (sum_s w_s o_part[s][row]) W_uv^g with w_s = exp(lse_s - lse),
+// lse = log sum_s exp(lse_s): the split-KV merge of the latent output and the
+// group's up-projection in one launch.  CTA: 64 rows of group g x the 128
+// outputs, 16 warps.  W_uv^g (128 KB) streams in through cp.async while the
+// warps merge the partials, 4 rows each with the loads of 4 splits in flight,
+// into a bf16 A tile in shared memory (the up-projection's operand is the
+// merged latent rounded to bf16); then 16 warps = 4 row blocks x 4 output
+// quarters of mma.sync tiles.
 constexpr int kLat = 512;
-
-__global__ void __launch_bounds__(256) combine_lat_kernel(int S, const float* __restrict__ o_part,
-                                                          const float* __restrict__ lse_part,
-                                                          bf16* __restrict__ o_lat, float* __restrict__ lse_out,
-                                                          long long rows) {
-  const long long wid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const long long row = wid >> 2;
-  const int q4 = (int)(wid & 3);
-  if (row >= rows) return;
-  float mx = -INFINITY;
-  for (int s = lane; s < S; s += 32) mx = fmaxf(mx, lse_part[(long long)s * rows + row]);
-  mx = warp_max(mx);
-  float Z = 0.f;
-  if (mx != -INFINITY)
-    for (int s = lane; s < S; s += 32) Z += expf(lse_part[(long long)s * rows + row] - mx);
-  Z = warp_sum(Z);
-  const float inv = mx == -INFINITY ? 0.f : 1.f / Z;
-  const int col = q4 * 128 + lane * 4;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (mx != -INFINITY) {
-    int s = 0;
-    for (; s + 4 <= S; s += 4) {
-      float4 v[4];
-      float w[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float ls = lse_part[(long long)(s + u) * rows + row];
-        w[u] = ls == -INFINITY ? 0.f : expf(ls - mx) * inv;
-        v[u] = *reinterpret_cast<const float4*>(o_part + ((long long)(s + u) * rows + row) * kLat + col);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc.x = fmaf(w[u], v[u].x, acc.x);
-        acc.y = fmaf(w[u], v[u].y, acc.y);
-        acc.z = fmaf(w[u], v[u].z, acc.z);
-        acc.w = fmaf(w[u], v[u].w, acc.w);
-      }
-    }
-    for (; s < S; ++s) {
-      const float ls = lse_part[(long long)s * rows + row];
-      const float w = ls == -INFINITY ? 0.f : expf(ls - mx) * inv;
-      const float4 v = *reinterpret_cast<const float4*>(o_part + ((long long)s * rows + row) * kLat + col);
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
-    }
-  }
-  *reinterpret_cast<uint2*>(o_lat + row * kLat + col) =
-      make_uint2(ptx::pack_bf16(acc.x, acc.y), ptx::pack_bf16(acc.z, acc.w));
-  if (q4 == 0 && lane == 0 && lse_out) lse_out[row] = mx == -INFINITY ? -INFINITY : mx + logf(Z);
-}
-
-// ------------------------------------------------------------- up_proj
-// out[row] = o_lat[row] W_uv^g.  CTA: 16 rows of group g x 128 outputs,
-// 4 warps of 32 outputs; the whole K = 512 of both operands is fetched with
-// cp.async in one go (A 16 KB, B 128 KB), so the GEMM pays one load latency.
-constexpr int kUpRows = 16, kUpN = 128;
+constexpr int kUpRows = 64, kUpN = 128, kUpThreads = 512;
 constexpr int kUpApitch = (kLat + 8) * 2;      // 1040 B
 constexpr int kUpBpitch = (kUpN + 8) * 2;      // 272 B
 constexpr int kUpAbytes = kUpRows * kUpApitch;
 constexpr int kUpBbytes = kLat * kUpBpitch;
 constexpr size_t kUpSmem = (size_t)kUpAbytes + kUpBbytes;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool pred) {
-  const int sz = pred ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-__global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict__ o_lat,
-                                                          const bf16* __restrict__ W_uv, bf16* __restrict__ out,
-                                                          int rows_g, int n_h, int m) {
+__global__ void __launch_bounds__(kUpThreads) merge_up_kernel(int S, const float* __restrict__ o_part,
+                                                              const float* __restrict__ lse_part,
+                                                              const bf16* __restrict__ W_uv, bf16* __restrict__ out,
+                                                              float* __restrict__ lse_out, long long rows,
+                                                              int rows_g, int n_h, int m) {
   extern __shared__ __align__(16) uint8_t sm[];
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,29 +137,78 @@ __global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict
     return lr < rows_g ? (long long)(lr / m) * n_h + g * m + lr % m : -1;
   };
   const bf16* Wg = W_uv + (size_t)g * kLat * kUpN;
-  for (int i = threadIdx.x; i < kUpRows * (kLat / 8); i += blockDim.x) {
-    const int rr = i / (kLat / 8), c = i % (kLat / 8);
-    const long long grow = grow_of(rr);
-    cp_async16(a + rr * kUpApitch + c * 16, o_lat + (grow < 0 ? 0 : grow) * kLat + c * 8, grow >= 0);
-  }
   for (int i = threadIdx.x; i < kLat * (kUpN / 8); i += blockDim.x) {
     const int kk = i / (kUpN / 8), c = i % (kUpN / 8);
     cp_async16(b + kk * kUpBpitch + c * 16, Wg + (size_t)kk * kUpN + c * 8, true);
   }
   cp_async_commit();
+
+  // merge: a warp per row, a lane on 4 columns of each 128-column quarter
+  for (int rr = warp; rr < kUpRows; rr += kUpThreads / 32) {
+    const long long row = grow_of(rr);
+    float4 acc[4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) acc[q4] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float mx = -INFINITY, Z = 0.f;
+    if (row >= 0) {
+      for (int s = lane; s < S; s += 32) mx = fmaxf(mx, lse_part[(long long)s * rows + row]);
+      mx = warp_max(mx);
+      if (mx != -INFINITY)
+        for (int s = lane; s < S; s += 32) Z += expf(lse_part[(long long)s * rows + row] - mx);
+      Z = warp_sum(Z);
+    }
+    if (mx != -INFINITY) {
+      const float inv = 1.f / Z;
+      for (int s0 = 0; s0 < S; s0 += 4) {
+        float w[4];
+        float4 v[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (s0 + u < S) {
+            const float ls = lse_part[(long long)(s0 + u) * rows + row];
+            w[u] = ls == -INFINITY ? 0.f : expf(ls - mx) * inv;
+            const float* src = o_part + ((long long)(s0 + u) * rows + row) * kLat + lane * 4;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) v[u][q4] = *reinterpret_cast<const float4*>(src + q4 * 128);
+          }
+        }
+        // the splits in order, as a sequential sum
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (s0 + u < S) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              acc[q4].x = fmaf(w[u], v[u][q4].x, acc[q4].x);
+              acc[q4].y = fmaf(w[u], v[u][q4].y, acc[q4].y);
+              acc[q4].z = fmaf(w[u], v[u][q4].z, acc[q4].z);
+              acc[q4].w = fmaf(w[u], v[u][q4].w, acc[q4].w);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+      *reinterpret_cast<uint2*>(sm + rr * kUpApitch + (q4 * 128 + lane * 4) * 2) =
+          make_uint2(ptx::pack_bf16(acc[q4].x, acc[q4].y), ptx::pack_bf16(acc[q4].z, acc[q4].w));
+    if (row >= 0 && lane == 0 && lse_out) lse_out[row] = mx == -INFINITY ? -INFINITY : mx + logf(Z);
+  }
   cp_async_wait0();
   __syncthreads();
+
+  // up-projection: warp = (16-row block, 32-output quarter)
+  const int wr = warp & 3, wn = warp >> 2;
   float acc[4][4];
 #pragma unroll
   for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 #pragma unroll 4
   for (int k0 = 0; k0 < kLat; k0 += 16) {
     uint32_t af[4];
-    ldsm_a(a, kUpApitch, 0, k0, af);
+    ldsm_a(a, kUpApitch, wr * 16, k0, af);
 #pragma unroll
     for (int np = 0; np < 2; ++np) {
       uint32_t bf[4];
-      ldsm_b_kn(b, kUpBpitch, warp * 32 + np * 16, k0, bf);
+      ldsm_b_kn(b, kUpBpitch, wn * 32 + np * 16, k0, bf);
       ptx::mma_bf16_16816(acc[2 * np], af, bf[0], bf[1]);
       ptx::mma_bf16_16816(acc[2 * np + 1], af, bf[2], bf[3]);
     }
@@ -216,11 +216,11 @@ __global__ void __launch_bounds__(128) up_proj_mma_kernel(const bf16* __restrict
   const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
-    const long long grow = grow_of(gid + 8 * h2);
+    const long long grow = grow_of(wr * 16 + gid + 8 * h2);
     if (grow < 0) continue;
 #pragma unroll
     for (int n = 0; n < 4; ++n)
-      *reinterpret_cast<uint32_t*>(out + grow * kUpN + warp * 32 + n * 8 + 2 * tig) =
+      *reinterpret_cast<uint32_t*>(out + grow * kUpN + wn * 32 + n * 8 + 2 * tig) =
           ptx::pack_bf16(acc[n][2 * h2], acc[n][2 * h2 + 1]);
   }
 }
@@ -239,7 +239,7 @@ cudaError_t absorb_q_mma(const Problem& p, const void* q, const void* W_uk, bf16
   cudaError_t e = ensure_smem_limit((const void*)absorb_q_mma_kernel, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((rows_g + kAqRows - 1) / kAqRows, d.r / kAqN, d.G);
-  absorb_q_mma_kernel<<<grid, 128, smem, s>>>((const bf16*)q, (const bf16*)W_uk, qt, rows_g, d.n_h, p.m, d.d_nope,
+  absorb_q_mma_kernel<<<grid, kAqThreads, smem, s>>>((const bf16*)q, (const bf16*)W_uk, qt, rows_g, d.n_h, p.m, d.d_nope,
                                               p.d_qk, d.r);
   count_launch();
   return cudaGetLastError();
@@ -250,18 +250,14 @@ bool gemm_combine_up_supports(const Problem& p) {
 }
 
 cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const float* lse_part, const void* W_uv,
-                           void* out, float* lse_out, bf16* o_lat, cudaStream_t s) {
+                           void* out, float* lse_out, cudaStream_t s) {
   const auto& d = p.d;
-  const long long warps = p.rows * 4;
-  combine_lat_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(S, o_part, lse_part, o_lat, lse_out, p.rows);
-  count_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   const int rows_g = p.ly.batch * d.s_q * p.m;
-  e = ensure_smem_limit((const void*)up_proj_mma_kernel, (int)kUpSmem);
+  cudaError_t e = ensure_smem_limit((const void*)merge_up_kernel, (int)kUpSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((rows_g + kUpRows - 1) / kUpRows, d.G);
-  up_proj_mma_kernel<<<grid, 128, kUpSmem, s>>>(o_lat, (const bf16*)W_uv, (bf16*)out, rows_g, d.n_h, p.m);
+  merge_up_kernel<<<grid, kUpThreads, kUpSmem, s>>>(S, o_part, lse_part, (const bf16*)W_uv, (bf16*)out, lse_out,
+                                                    p.rows, rows_g, d.n_h, p.m);
   count_launch();
   return cudaGetLastError();
 }

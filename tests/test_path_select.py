@@ -15,22 +15,22 @@ B200 = (148, 6559.0, 1656.2)   # SMs, copy GB/s, dense bf16 TFLOP/s (measured on
 # d = v = 128, B32, L 32K), measured on one B200 with `bench.py --sweep
 # crossover` (absorb ms, GQA ms).  A performance record, not an oracle value.
 MEASURED_B200 = {
-    (1, 1): (0.508, 0.153), (1, 2): (0.954, 0.256), (1, 4): (1.767, 0.463),
-    (2, 1): (0.506, 0.277), (2, 2): (0.953, 0.284), (2, 4): (1.768, 0.480),
-    (4, 1): (0.504, 0.485), (4, 2): (0.955, 0.516), (4, 4): (1.767, 0.538),
-    (8, 1): (0.506, 0.760), (8, 2): (0.954, 0.856), (8, 4): (1.769, 0.967),
-    (16, 1): (0.521, 1.513), (16, 2): (0.960, 1.512), (16, 4): (1.771, 1.624),
-    (32, 1): (0.513, 2.984), (32, 2): (0.981, 3.000), (32, 4): (1.771, 3.029),
-    (128, 1): (0.509, 12.188), (128, 2): (0.961, 12.174), (128, 4): (1.773, 12.187),
+    (1, 1): (0.512, 0.152), (1, 2): (0.933, 0.256), (1, 4): (1.735, 0.463),
+    (2, 1): (0.510, 0.277), (2, 2): (0.932, 0.283), (2, 4): (1.733, 0.480),
+    (4, 1): (0.511, 0.486), (4, 2): (0.933, 0.518), (4, 4): (1.734, 0.539),
+    (8, 1): (0.557, 0.765), (8, 2): (0.949, 0.862), (8, 4): (1.763, 0.972),
+    (16, 1): (0.519, 1.510), (16, 2): (0.970, 1.514), (16, 4): (1.772, 1.627),
+    (32, 1): (0.518, 2.989), (32, 2): (0.939, 3.003), (32, 4): (1.759, 3.028),
+    (128, 1): (0.502, 12.210), (128, 2): (0.936, 12.199), (128, 4): (1.736, 12.203),
 }
 
 # The DeepSeek-V3-shaped layer (n_h 128, G 16, B64) over context lengths,
 # `bench.py --sweep context` on the same B200: (L, s_q) -> (absorb ms, GQA ms).
 MEASURED_CONTEXT_B200 = {
-    (8192, 1): (0.310, 0.778), (8192, 2): (0.582, 0.804),
-    (16384, 1): (0.534, 1.507), (16384, 2): (1.014, 1.531),
-    (32768, 1): (0.972, 2.979), (32768, 2): (1.795, 3.003),
-    (65536, 1): (1.761, 5.970), (65536, 2): (3.354, 6.006),
+    (8192, 1): (0.280, 0.778), (8192, 2): (0.537, 0.804),
+    (16384, 1): (0.504, 1.510), (16384, 2): (0.949, 1.530),
+    (32768, 1): (0.944, 2.979), (32768, 2): (1.740, 3.001),
+    (65536, 1): (1.745, 5.971), (65536, 2): (3.372, 6.014),
 }
 
 
@@ -76,8 +76,8 @@ def test_structure_of_the_estimates(G):
     # the shared-RoPE K pool streams fewer bytes
     assert _est(G, 128, 16, 1, 64, 16384, shared=True)[2] < _est(G, 128, 16, 1, 64, 16384)[2]
     # doubling the context nearly doubles both (long-context regime); the
-    # absorbed call's side GEMMs and merge do not grow with L (measured: 0.534
-    # -> 0.972 ms, a factor 1.82)
+    # absorbed call's side GEMMs and merge do not grow with L (measured: 0.504
+    # -> 0.944 ms, a factor 1.87)
     p1, a1, g1 = _est(G, 128, 16, 1, 64, 16384)
     p2, a2, g2 = _est(G, 128, 16, 1, 64, 32768)
     assert 1.7 < a2 / a1 < 2.1 and 1.9 < g2 / g1 < 2.1
