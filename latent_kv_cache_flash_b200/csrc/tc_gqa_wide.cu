@@ -9,9 +9,13 @@
 //
 // One CTA per (key-range split, sequence, group, block of 128 rows):
 //  * the 128 x 192 query tile is stored into TMEM once (the A operand of
-//    the score MMAs), which leaves shared memory to a 4-stage mbarrier ring
-//    of 64-token K (64 x 192) and V (64 x 128) tiles (TMA, 2-D maps over the
-//    pools' token rows; a group's chunks are column offsets) and two P tiles;
+//    the score MMAs), which leaves shared memory to two mbarrier rings of
+//    64-token tiles (TMA, 2-D maps over the pools' token rows; a group's
+//    chunks are column offsets) and two P tiles: K tiles (64 x 192) in 3
+//    slots, each freed as soon as its score MMAs complete, and V tiles
+//    (64 x 128) in 7 slots, each held until its PV MMAs complete.  A tile's
+//    V lives about twice as long as its K (through the softmax), and with
+//    one ring for both the slots' lifetime bounded the tile rate;
 //  * warp 1 issues S = Q K^T (12 tcgen05.mma, M=128, N=64, K=16) into S[j % 2]
 //    in TMEM; warp 6 issues O[j % 2] += P[j % 2] V (4 tcgen05.mma, M=128,
 //    N=128, K=16, V as an MN-major operand);
@@ -38,13 +42,15 @@ constexpr int kDqk = 192;
 constexpr int kDv = 128;
 constexpr int kM = 128;                       // (query, head) rows per CTA
 constexpr int kT = 64;                        // tokens per tile
-constexpr int kStages = 4;
+constexpr int kKStages = 3, kVStages = 7;
 constexpr int kKChunks = kDqk / 64;           // 3 K chunks of 64 dims
 constexpr int kVChunks = kDv / 64;            // 2 V chunks
 constexpr int kChunkBytes = kT * 128;         // 8 KB
-constexpr int kStageBytes = (kKChunks + kVChunks) * kChunkBytes;   // 40 KB
+constexpr int kKSlotBytes = kKChunks * kChunkBytes;   // 24 KB
+constexpr int kVSlotBytes = kVChunks * kChunkBytes;   // 16 KB
 constexpr int kPBytes = kM * 128;             // 128 rows x 64 tokens (bf16)
-constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 2 * kPBytes + 2 * kM * 4 + 1024;
+constexpr size_t kSmemBytes =
+    (size_t)kKStages * kKSlotBytes + (size_t)kVStages * kVSlotBytes + 2 * kPBytes + 2 * kM * 4 + 1024;
 constexpr uint32_t kTmemCols = 512;           // S: 2 x 64 at 0, O: 2 x 128 at 128, Q: 96 at 384
 constexpr uint32_t kSCol = 0, kOCol = 128, kQCol = 384;
 constexpr int kThreads = 12 * 32;
@@ -71,12 +77,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const WideParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sKV = smem;
-  uint8_t* sP = sKV + kStages * kStageBytes;           // P[2]: one per softmax group
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + kKStages * kKSlotBytes;
+  uint8_t* sP = sV + kVStages * kVSlotBytes;           // P[2]: one per softmax group
   float* sML = reinterpret_cast<float*>(sP + 2 * kPBytes);   // the odd group's row max and sum
   __shared__ __align__(8) uint64_t q_full, qk_drain, pv_drain;
-  __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], p_full[2],
-      pv_done[2];
+  __shared__ __align__(8) uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages],
+      s_full[2], s_free[2], p_full[2], pv_done[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -90,9 +97,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(&q_full, 4);
     ptx::mbar_init(&qk_drain, 1);
     ptx::mbar_init(&pv_drain, 1);
-    for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(&kv_full[s], 2);
-      ptx::mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < kKStages; ++s) {
+      ptx::mbar_init(&k_full[s], 1);
+      ptx::mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      ptx::mbar_init(&v_full[s], 1);
+      ptx::mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&s_full[s], 1);
@@ -119,57 +130,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 || warp == 7) {
     // ---------------------------------------------------- TMA producers
     // One issuing thread brings about 27 bytes per cycle into an SM; the
-    // tile needs more at the tensor pipe's pace, so warp 0 loads the K
-    // chunks and warp 7 the V chunks, both arriving on the stage's barrier.
+    // tile needs more at the tensor pipe's pace, so warp 0 loads the K ring
+    // and warp 7 the V ring.
     const bool kside = warp == 0;
+    const int nst = kside ? kKStages : kVStages;
+    uint64_t* full = kside ? k_full : v_full;
+    uint64_t* empty = kside ? k_empty : v_empty;
     if (lane == 0 && n_tiles > 0) {
-      ptx::prefetch_tmap(&kmap);
-      ptx::prefetch_tmap(&vmap);
+      ptx::prefetch_tmap(kside ? &kmap : &vmap);
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kStages, k = j / kStages;
-        if (k > 0 && !ptx::mbar_wait(&kv_empty[s], (k - 1) & 1)) {
+        const int s = j % nst, k = j / nst;
+        if (k > 0 && !ptx::mbar_wait(&empty[s], (k - 1) & 1)) {
           flag_status(p.st, GQLA_DEV_TIMEOUT);
           atomicExch(&abort_flag, 1);
           break;
         }
         if (*(volatile int*)&abort_flag) break;
         const int row0 = (int)token_row(p.ly, b, t_begin + j * kT, nullptr);
-        uint8_t* dst = sKV + s * kStageBytes;
         if (kside) {
-          ptx::mbar_arrive_expect_tx(&kv_full[s], kKChunks * kChunkBytes);
-          ptx::tma_load_2d(dst, &kmap, &kv_full[s], p.kr.nope_at(g), row0);
-          ptx::tma_load_2d(dst + kChunkBytes, &kmap, &kv_full[s], p.kr.nope_at(g) + 64, row0);
-          ptx::tma_load_2d(dst + 2 * kChunkBytes, &kmap, &kv_full[s], p.kr.rope_at(g), row0);
+          uint8_t* dst = sK + s * kKSlotBytes;
+          ptx::mbar_arrive_expect_tx(&full[s], kKSlotBytes);
+          ptx::tma_load_2d(dst, &kmap, &full[s], p.kr.nope_at(g), row0);
+          ptx::tma_load_2d(dst + kChunkBytes, &kmap, &full[s], p.kr.nope_at(g) + 64, row0);
+          ptx::tma_load_2d(dst + 2 * kChunkBytes, &kmap, &full[s], p.kr.rope_at(g), row0);
         } else {
-          ptx::mbar_arrive_expect_tx(&kv_full[s], kVChunks * kChunkBytes);
+          uint8_t* dst = sV + s * kVSlotBytes;
+          ptx::mbar_arrive_expect_tx(&full[s], kVSlotBytes);
           for (int c = 0; c < kVChunks; ++c)
-            ptx::tma_load_2d(dst + (kKChunks + c) * kChunkBytes, &vmap, &kv_full[s], g * kDv + 64 * c, row0);
+            ptx::tma_load_2d(dst + c * kChunkBytes, &vmap, &full[s], g * kDv + 64 * c, row0);
         }
         issued = j + 1;
       }
-      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-        ptx::mbar_wait(&kv_full[j % kStages], (j / kStages) & 1);
+      // no copy may be in flight when the CTA exits
+      for (int j = issued > nst ? issued - nst : 0; j < issued; ++j) ptx::mbar_wait(&full[j % nst], (j / nst) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------- QK issuer, TMEM owner
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = ptx::idesc_bf16(kM, kT, false, false);
-      const uint32_t kv_addr = ptx::smem_u32(sKV);
+      const uint32_t k_addr = ptx::smem_u32(sK);
       bool ok = ptx::mbar_wait(&q_full, 0);
       ptx::tc_fence_after();
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kStages, sb = j & 1;
-        ok = ptx::mbar_wait(&kv_full[s], (j / kStages) & 1);
+        const int s = j % kKStages, sb = j & 1;
+        ok = ptx::mbar_wait(&k_full[s], (j / kKStages) & 1);
         if (ok && j >= 2) ok = ptx::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint64_t bd0 = ptx::umma_desc_sw128(kv_addr + s * kStageBytes, 16, 1024);
+        const uint64_t bd0 = ptx::umma_desc_sw128(k_addr + s * kKSlotBytes, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < kDqk / 16; ++kk)
           ptx::umma_bf16_ts(tmem + kSCol + (uint32_t)kT * sb, tmem + kQCol + 8u * kk,
                             ptx::umma_desc_add(bd0, (kk >> 2) * kChunkBytes + (kk & 3) * 32), idesc_qk, kk > 0);
         ptx::umma_commit(&s_full[sb]);
+        ptx::umma_commit(&k_empty[s]);            // the K slot is free once these MMAs complete
       }
       if (!ok) {
         flag_status(p.st, GQLA_DEV_TIMEOUT);
@@ -182,21 +197,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- PV issuer
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_pv = ptx::idesc_bf16(kM, kDv, false, true);
-      const uint32_t kv_addr = ptx::smem_u32(sKV);
+      const uint32_t v_addr = ptx::smem_u32(sV);
       const uint64_t ad0 = ptx::umma_desc_sw128(ptx::smem_u32(sP), 16, 1024);
       bool ok = true;
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kStages, sb = j & 1;
+        const int s = j % kVStages, sb = j & 1;
         ok = ptx::mbar_wait(&p_full[sb], (j >> 1) & 1);
+        if (ok) ok = ptx::mbar_wait(&v_full[s], (j / kVStages) & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint64_t bd0 = ptx::umma_desc_sw128(kv_addr + s * kStageBytes + kKChunks * kChunkBytes, kChunkBytes, 1024);
+        const uint64_t bd0 = ptx::umma_desc_sw128(v_addr + s * kVSlotBytes, kChunkBytes, 1024);
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
           ptx::umma_bf16(tmem + kOCol + (uint32_t)kDv * sb, ptx::umma_desc_add(ad0, sb * kPBytes + kk * 32),
                          ptx::umma_desc_add(bd0, kk * 16 * 128), idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
         ptx::umma_commit(&pv_done[sb]);
-        ptx::umma_commit(&kv_empty[s]);
+        ptx::umma_commit(&v_empty[s]);
       }
       if (!ok) {
         flag_status(p.st, GQLA_DEV_TIMEOUT);
@@ -244,7 +260,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int last = -1;                               // this group's last tile
     for (int j = gp; j < n_tiles; j += 2) {
-      const int s = j % kStages;
       const int t0 = t_begin + j * kT;
       last = j;
       if (ok) ok = ptx::mbar_wait(&s_full[gp], (j >> 1) & 1);
@@ -352,14 +367,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l_sum += acc;
       if (t0 + kT > L) {
-        // value rows past the sequence may hold anything: zero them for PV
+        // value rows past the sequence may hold anything: zero them for PV,
+        // once the tile's V has landed (its slot cannot be refilled before
+        // this group's P is delivered)
+        const int sv = j % kVStages;
+        bool vok = ok && ptx::mbar_wait(&v_full[sv], (j / kVStages) & 1);
+        vok = __all_sync(0xffffffffu, vok);
         const int tid = 32 * qd + lane;
-        for (int idx = tid; idx < kT * kVChunks * 8; idx += 128) {
+        for (int idx = tid; vok && idx < kT * kVChunks * 8; idx += 128) {
           const int tok = idx / (kVChunks * 8), rem = idx % (kVChunks * 8);
           if (t0 + tok >= L)
-            *reinterpret_cast<uint4*>(sKV + s * kStageBytes + (kKChunks + rem / 8) * kChunkBytes +
-                                      ptx::swz128(tok, rem % 8)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sV + sv * kVSlotBytes + (rem / 8) * kChunkBytes + ptx::swz128(tok, rem % 8)) =
+                make_uint4(0, 0, 0, 0);
         }
+        ok = vok;
       }
       ptx::fence_proxy_async_smem();
       asm volatile("bar.sync %0, 128;" ::"r"(1 + gp) : "memory");   // the tail zeroing is shared by the group
