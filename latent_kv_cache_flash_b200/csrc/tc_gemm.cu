@@ -109,20 +109,21 @@ __global__ void __launch_bounds__(kAqThreads) absorb_q_mma_kernel(const bf16* __
 // ------------------------------------------------------------ merge_up
 // out[row] = (sum_s w_s o_part[s][row]) W_uv^g with w_s = exp(lse_s - lse),
 // lse = log sum_s exp(lse_s): the split-KV merge of the latent output and the
-// group's up-projection in one launch.  CTA: 64 rows of group g x the 128
-// outputs, 16 warps.  W_uv^g (128 KB) streams in through cp.async while the
-// warps merge the partials, 4 rows each with the loads of 4 splits in flight,
-// into a bf16 A tile in shared memory (the up-projection's operand is the
-// merged latent rounded to bf16); then 16 warps = 4 row blocks x 4 output
-// quarters of mma.sync tiles.
+// group's up-projection in one launch.  CTA: R rows of group g (64, or 32
+// or 16 when fewer CTAs would leave SMs idle) x the 128 outputs, 16 warps.
+// W_uv^g (128 KB) streams in through cp.async while the warps merge the
+// partials, R/16 rows each with the loads of 4 splits in flight, into a bf16
+// A tile in shared memory (the up-projection's operand is the merged latent
+// rounded to bf16); then R/16 row blocks x 4 output quarters of mma.sync
+// tiles, one warp each.
 constexpr int kLat = 512;
-constexpr int kUpRows = 64, kUpN = 128, kUpThreads = 512;
+constexpr int kUpN = 128, kUpThreads = 512;
 constexpr int kUpApitch = (kLat + 8) * 2;      // 1040 B
 constexpr int kUpBpitch = (kUpN + 8) * 2;      // 272 B
-constexpr int kUpAbytes = kUpRows * kUpApitch;
 constexpr int kUpBbytes = kLat * kUpBpitch;
-constexpr size_t kUpSmem = (size_t)kUpAbytes + kUpBbytes;
+constexpr size_t up_smem(int rows) { return (size_t)rows * kUpApitch + kUpBbytes; }
 
+template <int kUpRows>
 __global__ void __launch_bounds__(kUpThreads) merge_up_kernel(int S, const float* __restrict__ o_part,
                                                               const float* __restrict__ lse_part,
                                                               const bf16* __restrict__ W_uv, bf16* __restrict__ out,
@@ -131,7 +132,7 @@ __global__ void __launch_bounds__(kUpThreads) merge_up_kernel(int S, const float
   extern __shared__ __align__(16) uint8_t sm[];
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t a = ptx::smem_u32(sm), b = a + kUpAbytes;
+  const uint32_t a = ptx::smem_u32(sm), b = a + kUpRows * kUpApitch;
   auto grow_of = [&](int rr) -> long long {
     const int lr = blockIdx.x * kUpRows + rr;
     return lr < rows_g ? (long long)(lr / m) * n_h + g * m + lr % m : -1;
@@ -197,7 +198,9 @@ __global__ void __launch_bounds__(kUpThreads) merge_up_kernel(int S, const float
   __syncthreads();
 
   // up-projection: warp = (16-row block, 32-output quarter)
-  const int wr = warp & 3, wn = warp >> 2;
+  constexpr int kRb = kUpRows / 16;
+  if (warp >= 4 * kRb) return;
+  const int wr = warp % kRb, wn = warp / kRb;
   float acc[4][4];
 #pragma unroll
   for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -253,11 +256,25 @@ cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const f
                            void* out, float* lse_out, cudaStream_t s) {
   const auto& d = p.d;
   const int rows_g = p.ly.batch * d.s_q * p.m;
-  cudaError_t e = ensure_smem_limit((const void*)merge_up_kernel, (int)kUpSmem);
+  // the largest row tile that still gives about a CTA per SM: the merge of a
+  // CTA's rows is bound by its loads in flight, so small batches take more
+  // CTAs of fewer rows (each loads W_uv^g from L2)
+  auto ctas = [&](int rows) { return (long long)((rows_g + rows - 1) / rows) * d.G; };
+  const int want = num_sms() * 4 / 5;
+  const int R = ctas(64) >= want ? 64 : ctas(32) >= want ? 32 : 16;
+  const void* fn = R == 64 ? (const void*)merge_up_kernel<64>
+                 : R == 32 ? (const void*)merge_up_kernel<32> : (const void*)merge_up_kernel<16>;
+  cudaError_t e = ensure_smem_limit(fn, (int)up_smem(R));
   if (e != cudaSuccess) return e;
-  dim3 grid((rows_g + kUpRows - 1) / kUpRows, d.G);
-  merge_up_kernel<<<grid, kUpThreads, kUpSmem, s>>>(S, o_part, lse_part, (const bf16*)W_uv, (bf16*)out, lse_out,
-                                                    p.rows, rows_g, d.n_h, p.m);
+  dim3 grid((rows_g + R - 1) / R, d.G);
+  const bf16* w = (const bf16*)W_uv;
+  bf16* o = (bf16*)out;
+  if (R == 64)
+    merge_up_kernel<64><<<grid, kUpThreads, up_smem(64), s>>>(S, o_part, lse_part, w, o, lse_out, p.rows, rows_g, d.n_h, p.m);
+  else if (R == 32)
+    merge_up_kernel<32><<<grid, kUpThreads, up_smem(32), s>>>(S, o_part, lse_part, w, o, lse_out, p.rows, rows_g, d.n_h, p.m);
+  else
+    merge_up_kernel<16><<<grid, kUpThreads, up_smem(16), s>>>(S, o_part, lse_part, w, o, lse_out, p.rows, rows_g, d.n_h, p.m);
   count_launch();
   return cudaGetLastError();
 }
