@@ -26,7 +26,7 @@ constexpr double kDefaultTcTflops = 1656.2;
 constexpr double kEtaStream = 1.08;     // GQA mma.sync kernel, <= 16 rows a group: K/V read stream (1.07..1.10 of the copy rate)
 constexpr double kEtaStreamWide = 1.0;  // the same kernel at 17..63 rows a group, where its MMAs slow each CTA's stream
 constexpr double kEtaWideTc = 0.54;     // GQA tcgen05 kernel: a 128-row block-tile, full or not (softmax-bound)
-constexpr double kEtaWideBw = 0.94;     // its K/V stream, paid by the first row block of a tile (the others hit L2)
+constexpr double kEtaWideBw = 1.0;      // its K/V stream, paid by the first row block of a tile (the others hit L2)
 constexpr double kWideCtaUs = 11.0;     // its CTA prologue (query into TMEM) + epilogue (merge of two states, output)
 constexpr double kEtaAbsorbTc = 0.42;   // absorb tcgen05 kernel: M=64 tiles, N=64 score MMAs
 constexpr double kEtaAbsorbBw = 0.90;   // a CTA's latent tile loads (every row block loads each tile into its SM)

@@ -68,6 +68,22 @@ def test_bf16_dsv3_shapes(s_q, path):
     H.check_units(inp, out, lse, H.sample_units(inp, 8), "dsv3 bf16 %s s_q=%d" % (path, s_q))
 
 
+@pytest.mark.parametrize("B", [5, 33, 61])
+def test_bf16_absorb_merge_row_tiles(B):
+    """The absorbed call's split merge and up-projection take 16, 32 or 64
+    rows of a group per CTA, the largest that still fills the SMs: at G 16
+    (8 rows a group per token) B 5 takes 16-row tiles, B 33 32-row tiles with
+    a ragged last tile, B 61 64-row tiles with a ragged last tile.  Three
+    splits, so every row merges several partials."""
+    d = synth.Dims(**DSV3, s_q=1)
+    g = torch.Generator()
+    g.manual_seed(B)
+    lens = torch.randint(200, 700, (B,), generator=g).tolist()
+    inp = _wl(d, B, lens, seed=B)
+    out, lse = H.run_decode(inp, "absorb", num_splits=3)
+    H.check_units(inp, out, lse, H.sample_units(inp, 6, seed=B), "absorb merge tiles B=%d" % B)
+
+
 @pytest.mark.parametrize("G", [1, 2, 4, 32, 128])
 @pytest.mark.parametrize("s_q", [1, 4])
 def test_bf16_group_counts(G, s_q):
