@@ -117,7 +117,7 @@ SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, 
     }
     return plan_of(best_s);
   }
-  long long units, slots;
+  long long units, slots, rb = 1;
   double unit_bytes, part_bytes, cta_tokens;
   if (path == GQLA_PATH_ABSORB) {
     units = (long long)l.batch * ((d.n_h * d.s_q + 63) / 64);
@@ -126,21 +126,40 @@ SplitPlan make_plan(const gqla_dims& d, const gqla_kv_layout& l, int requested, 
     part_bytes = (double)rows * (d.r + 1) * 4 * 2;
     cta_tokens = 300.0;
   } else {
-    // the tcgen05 GQA kernel: 128-row blocks, one CTA per SM
-    units = (long long)l.batch * d.G * (((d.n_h / d.G) * d.s_q + 127) / 128);
+    // the tcgen05 GQA kernel: 128-row blocks, one CTA per SM.  Its CTA costs
+    // about 900 tokens of stream up front (the first tile's latency, the
+    // query into TMEM, the merge of the two softmax states).  Only the first
+    // row block of a (sequence, group, split) reads a K/V tile from HBM (the
+    // others hit L2), and about 95% of the SMs' worth of such readers keep
+    // HBM busy: a wave with more of them streams each tile proportionally
+    // slower.  (Measured on B200, n_h 128, B32 L32K: one wave of 128 CTAs,
+    // 1-4 splits, beats two to seven waves of 8-9 splits by 4-15% at every
+    // shape with 64-512 rows a group.)
+    rb = ((d.n_h / d.G) * d.s_q + 127) / 128;
+    units = (long long)l.batch * d.G * rb;
     slots = (long long)num_sms();
     unit_bytes = 2.0 * (d.d_nope + d.d_rope + d.d_v);
     part_bytes = (double)rows * (d.d_v + 1) * 4 * 2;
-    cta_tokens = 0.0;
+    cta_tokens = 900.0;
   }
+  const double busy = 0.95 * (double)slots;
   long long best_s = 1;
   double best = -1.0;
   for (long long S = 1; S <= max_s; ++S) {
     const long long c = chunk_for(S);
     const long long Se = (L + c - 1) / c;
     if (Se != S) continue;
-    const long long waves = (units * Se + slots - 1) / slots;
-    const double cost = (double)waves * (c + cta_tokens) * unit_bytes * slots + (Se > 1 ? Se * part_bytes : 0.0);
+    double cost = Se > 1 ? Se * part_bytes : 0.0;
+    if (path == GQLA_PATH_ABSORB) {
+      const long long waves = (units * Se + slots - 1) / slots;
+      cost += (double)waves * (c + cta_tokens) * unit_bytes * slots;
+    } else {
+      for (long long left = units * Se; left > 0; left -= slots) {
+        const double w = (double)(left < slots ? left : slots);
+        const double share = w / (double)rb / busy;
+        cost += (c + cta_tokens) * unit_bytes * slots * (share > 1.0 ? share : 1.0);
+      }
+    }
     if (best < 0 || cost < best * 0.999) {
       best = cost;
       best_s = Se;

@@ -25,8 +25,8 @@ constexpr double kDefaultTcTflops = 1656.2;
 // L 8K..64K):
 constexpr double kEtaStream = 1.08;     // GQA mma.sync kernel, <= 16 rows a group: K/V read stream (1.07..1.10 of the copy rate)
 constexpr double kEtaStreamWide = 1.0;  // the same kernel at 17..63 rows a group, where its MMAs slow each CTA's stream
-constexpr double kEtaWideTc = 0.54;     // GQA tcgen05 kernel: a 128-row block-tile, full or not (softmax-bound)
-constexpr double kEtaWideBw = 1.0;      // its K/V stream, paid by the first row block of a tile (the others hit L2)
+constexpr double kEtaWideTc = 0.60;     // GQA tcgen05 kernel: a 128-row block-tile, full or not (softmax-bound)
+constexpr double kEtaWideBw = 0.98;     // its K/V stream: a wave's first row blocks share HBM (the others hit L2)
 constexpr double kWideCtaUs = 11.0;     // its CTA prologue (query into TMEM) + epilogue (merge of two states, output)
 constexpr double kEtaAbsorbTc = 0.42;   // absorb tcgen05 kernel: M=64 tiles, N=64 score MMAs
 constexpr double kEtaAbsorbBw = 0.90;   // a CTA's latent tile loads (every row block loads each tile into its SM)
@@ -73,12 +73,20 @@ double gqa_us(const Problem& p, long long T, const Rates& r) {
   const double tiles = (double)T / 64.0 + 0.5 * p.ly.batch;
   double dec;
   if (tc_gqa_wide_supports(p)) {
+    // per wave: each CTA's tiles at the tensor rate, or at the wave's share
+    // of HBM (only the first row block of a tile reads it from HBM)
     const long long rb = (p.m * d.s_q + 127) / 128;
     const double flops_tile = 2.0 * 128 * 64 * (p.d_qk + d.d_v);
-    const double bytes_tile = 64.0 * row_bytes / d.G / rb;
-    const double t_tile = fmax(flops_tile / (r.tc_sm * kEtaWideTc), bytes_tile / (r.bw_sm * kEtaWideBw));
+    const double bytes_tile = 64.0 * row_bytes / d.G;
+    const double t_tc = flops_tile / (r.tc_sm * kEtaWideTc);
     const double ctas = (double)p.ly.batch * d.G * p.plan.num_splits * rb;
-    dec = ceil(ctas / r.sms) * (kWideCtaUs + tiles * d.G * rb / ctas * t_tile);
+    const double tiles_cta = tiles * d.G * rb / ctas;
+    dec = 0.0;
+    for (double left = ctas; left > 0.0; left -= r.sms) {
+      const double w = fmin(left, (double)r.sms);
+      const double t_hbm = w / rb * bytes_tile / (r.bw * kEtaWideBw);
+      dec += kWideCtaUs + tiles_cta * fmax(t_tc, t_hbm);
+    }
   } else {
     dec = (double)T * row_bytes / (r.bw * (p.m * d.s_q <= 16 ? kEtaStream : kEtaStreamWide));
   }

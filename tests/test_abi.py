@@ -179,6 +179,32 @@ def test_plan_matches_the_measured_best_split_counts(G, shape):
     assert got == MEASURED_PLANS[shape]
 
 
+# The tcgen05 GQA kernel (64+ rows a group) on the crossover grid (n_h 128,
+# B32, L32K): every split count timed on one B200 (GQA call, us), the best
+# count per shape.  One wave of 128 CTAs beats several waves of smaller
+# chunks wherever the wave's HBM-reading CTAs already keep HBM busy.
+MEASURED_WIDE_PLANS = {
+    (1, 1): 4,    # 4: 127.9; 8: 146.6; 9: 145.6
+    (2, 1): 2,    # 2: 238.3; 4: 250.7; 9: 258.0
+    (2, 2): 2,    # 2: 245.7; 4: 257.7; 9: 279.8
+    (4, 2): 1,    # 1: 479.0; 2: 502.0; 8: 545.8
+    (1, 2): 2,    # 2: 238.3; 4: 249.0; 9: 256.1
+    (1, 4): 1,    # 1: 446.6; 2: 462.6; 8: 504.8
+    (4, 4): 1,    # 1: 466.1; 2: 495.9; 8: 590.7
+    (8, 4): 4,    # 4: 897.8 (first timed) / 1000.5; 1: 923.7; 2: 1103.4
+}
+
+
+@pytest.mark.parametrize("shape", sorted(MEASURED_WIDE_PLANS))
+def test_wide_gqa_plan_matches_the_measured_best(G, shape):
+    from latent_kv_cache_flash_b200 import synth
+    groups, s_q = shape
+    d = G.make_dims(synth.Dims(n_h=128, G=groups, d_nope=128, d_rope=64, d_v=128, r=512, s_q=s_q))
+    lens = torch.full((32,), 32768, dtype=torch.int32)
+    lay = G.make_layout(lens, 32768, 0, 32768)
+    assert G.gqla_num_splits(d, lay, 0, G.GQLA_PATH_GQA) == MEASURED_WIDE_PLANS[shape]
+
+
 def test_plan_splits_small_batches_to_fill_the_gpu(G):
     from latent_kv_cache_flash_b200 import synth
     d = G.make_dims(synth.Dims(n_h=32, G=8, d_nope=128, d_rope=64, d_v=128, r=512))

@@ -15,22 +15,22 @@ B200 = (148, 6559.0, 1656.2)   # SMs, copy GB/s, dense bf16 TFLOP/s (measured on
 # d = v = 128, B32, L 32K), measured on one B200 with `bench.py --sweep
 # crossover` (absorb ms, GQA ms).  A performance record, not an oracle value.
 MEASURED_B200 = {
-    (1, 1): (0.494, 0.149), (1, 2): (0.935, 0.252), (1, 4): (1.735, 0.466),
-    (2, 1): (0.492, 0.254), (2, 2): (0.934, 0.273), (2, 4): (1.735, 0.473),
-    (4, 1): (0.493, 0.484), (4, 2): (0.934, 0.477), (4, 4): (1.737, 0.516),
-    (8, 1): (0.492, 0.745), (8, 2): (0.935, 0.852), (8, 4): (1.738, 0.887),
-    (16, 1): (0.496, 1.482), (16, 2): (0.940, 1.489), (16, 4): (1.737, 1.605),
-    (32, 1): (0.504, 2.941), (32, 2): (0.940, 2.951), (32, 4): (1.744, 2.980),
-    (128, 1): (0.503, 11.885), (128, 2): (0.939, 11.888), (128, 4): (1.747, 11.909),
+    (1, 1): (0.493, 0.130), (1, 2): (0.938, 0.227), (1, 4): (1.738, 0.414),
+    (2, 1): (0.494, 0.236), (2, 2): (0.938, 0.235), (2, 4): (1.738, 0.416),
+    (4, 1): (0.493, 0.485), (4, 2): (0.938, 0.440), (4, 4): (1.739, 0.448),
+    (8, 1): (0.492, 0.747), (8, 2): (0.938, 0.852), (8, 4): (1.743, 0.861),
+    (16, 1): (0.502, 1.486), (16, 2): (0.938, 1.488), (16, 4): (1.738, 1.603),
+    (32, 1): (0.495, 2.938), (32, 2): (0.936, 2.950), (32, 4): (1.737, 2.978),
+    (128, 1): (0.501, 11.867), (128, 2): (0.939, 11.873), (128, 4): (1.738, 11.879),
 }
 
 # The DeepSeek-V3-shaped layer (n_h 128, G 16, B64) over context lengths,
 # `bench.py --sweep context` on the same B200: (L, s_q) -> (absorb ms, GQA ms).
 MEASURED_CONTEXT_B200 = {
-    (8192, 1): (0.279, 0.770), (8192, 2): (0.535, 0.793),
-    (16384, 1): (0.506, 1.486), (16384, 2): (0.951, 1.509),
-    (32768, 1): (0.945, 2.928), (32768, 2): (1.745, 2.950),
-    (65536, 1): (1.745, 5.857), (65536, 2): (3.330, 5.885),
+    (8192, 1): (0.278, 0.770), (8192, 2): (0.532, 0.793),
+    (16384, 1): (0.504, 1.485), (16384, 2): (0.953, 1.509),
+    (32768, 1): (0.946, 2.928), (32768, 2): (1.743, 2.953),
+    (65536, 1): (1.740, 5.852), (65536, 2): (3.326, 5.877),
 }
 
 
@@ -76,8 +76,8 @@ def test_structure_of_the_estimates(G):
     # the shared-RoPE K pool streams fewer bytes
     assert _est(G, 128, 16, 1, 64, 16384, shared=True)[2] < _est(G, 128, 16, 1, 64, 16384)[2]
     # doubling the context nearly doubles both (long-context regime); the
-    # absorbed call's side GEMMs and merge do not grow with L (measured: 0.506
-    # -> 0.945 ms, a factor 1.87)
+    # absorbed call's side GEMMs and merge do not grow with L (measured: 0.504
+    # -> 0.946 ms, a factor 1.88)
     p1, a1, g1 = _est(G, 128, 16, 1, 64, 16384)
     p2, a2, g2 = _est(G, 128, 16, 1, 64, 32768)
     assert 1.7 < a2 / a1 < 2.1 and 1.9 < g2 / g1 < 2.1
