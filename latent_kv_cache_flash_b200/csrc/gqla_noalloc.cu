@@ -27,32 +27,37 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 // primary context loads the module afresh, so a changed context triggers a
 // new lookup instead of reusing a stale address.
 typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// The driver's cuCtxGetCurrent, looked up once through the runtime (the
-// library does not link libcuda).
-CtxGetCurrentFn ctx_get_current_fn() {
-  static CtxGetCurrentFn fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (CtxGetCurrentFn)f;
+// A driver entry point, looked up through the runtime (the library does not
+// link libcuda); nullptr when the driver lacks it.
+void* driver_fn(const char* name) {
+  void* f = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return fn;
+  return f;
 }
 
-CUcontext current_context() {
-  CtxGetCurrentFn fn = ctx_get_current_fn();
+// An identity of the context current on this thread, 0 when there is none:
+// the driver's unique context id (never reused within the process), else the
+// context handle.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = (CtxGetCurrentFn)driver_fn("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = (CtxGetIdFn)driver_fn("cuCtxGetId");
   CUcontext ctx = nullptr;
-  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
-  return ctx;
+  if (!get_current || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id && get_id(ctx, &id) == CUDA_SUCCESS && id != 0) return id;
+  return (unsigned long long)(uintptr_t)ctx;
 }
 
 void* scratch_for_current_device(gqla_status* status) {
   static std::mutex mu;
   static void* cached[64] = {nullptr};
-  static CUcontext cached_ctx[64] = {nullptr};
+  static unsigned long long cached_ctx[64] = {0};
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
@@ -61,13 +66,13 @@ void* scratch_for_current_device(gqla_status* status) {
   }
   // the context current on this thread (none before the runtime's first call
   // here; the symbol lookup below creates the device's primary context then)
-  CUcontext ctx = current_context();
+  unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (ctx != nullptr && cached[dev] != nullptr && cached_ctx[dev] == ctx) return cached[dev];
+  if (ctx != 0 && cached[dev] != nullptr && cached_ctx[dev] == ctx) return cached[dev];
   void* ptr = nullptr;
   const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-  if (e == cudaSuccess) ctx = current_context();
-  if (e != cudaSuccess || ptr == nullptr || ctx == nullptr) {
+  if (e == cudaSuccess) ctx = current_context_id();
+  if (e != cudaSuccess || ptr == nullptr || ctx == 0) {
     cudaGetLastError();
     cached[dev] = nullptr;
     *status = GQLA_ERR_CUDA;
