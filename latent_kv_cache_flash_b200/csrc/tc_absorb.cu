@@ -27,7 +27,9 @@
 //    is rescaled only when a row maximum grows by more than 2^8, through the
 //    same shape so the Q~/S lanes are never touched), write P (bf16) to shared
 //    memory, and at the end stage O through shared memory to write the fp32
-//    latent output and the log-sum-exp of the split.
+//    latent output and the log-sum-exp of the split;
+//  * warps 0 and 7 load the latent tiles, five and four of a tile's nine
+//    128-byte column chunks, onto the stage's barrier.
 #include <math.h>
 
 #include "ptx.cuh"
@@ -55,7 +57,7 @@ constexpr uint32_t kQCols = kE / 2;                  // 288 columns of bf16 pair
 constexpr uint32_t kSCol = kQCols;                   // S buffers at 288 and 352
 constexpr uint32_t kOLane = 16u << 16;               // O in lanes 16-31 of each quarter
 constexpr int kOStride = kR + 4;                     // staging pitch (floats) for the output
-constexpr int kThreads = 7 * 32;
+constexpr int kThreads = 8 * 32;
 constexpr float kRescaleLog2 = 8.f;
 
 static_assert(kSCol + 2 * kTk <= kTmemCols, "Q~ and the S buffers must fit the low half-lanes");
@@ -99,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(&qk_drain, 1);
     ptx::mbar_init(&pv_drain, 1);
     for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(&kv_full[s], 1);
+      ptx::mbar_init(&kv_full[s], 2);
       ptx::mbar_init(&kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -123,8 +125,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = t_stop > t_begin ? (t_stop - t_begin + kTk - 1) / kTk : 0;
   const long long grow0 = (long long)b * p.rows_unit + (long long)hb * kM;
 
-  if (warp == 0) {
-    // ------------------------------------------------------- TMA producer
+  if (warp == 0 || warp == 7) {
+    // ------------------------------------------------------- TMA producers
+    // One issuing thread brings at most about 27 bytes per cycle into the SM,
+    // so a 72 KB tile took about 2.7k cycles to land, inside the loop through
+    // the 3-stage ring; two threads (chunks 0-4 and 5-8) halve that.
+    const int c_lo = warp == 0 ? 0 : 5, c_hi = warp == 0 ? 5 : kChunks;
     if (lane == 0 && n_tiles > 0) {
       ptx::prefetch_tmap(&kv_map);
       int issued = 0;
@@ -138,8 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*(volatile int*)&abort_flag) break;
         const int row0 = (int)token_row(p.ly, b, t_begin + j * kTk, nullptr);
         uint8_t* dst = sKV + s * kStageBytes;
-        ptx::mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
-        for (int c = 0; c < kChunks; ++c) ptx::tma_load_2d(dst + c * kKVChunk, &kv_map, &kv_full[s], 64 * c, row0);
+        ptx::mbar_arrive_expect_tx(&kv_full[s], (c_hi - c_lo) * kKVChunk);
+        for (int c = c_lo; c < c_hi; ++c) ptx::tma_load_2d(dst + c * kKVChunk, &kv_map, &kv_full[s], 64 * c, row0);
         issued = j + 1;
       }
       // no copy may still be landing in shared memory when the CTA retires
