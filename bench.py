@@ -19,7 +19,7 @@ of one step).  The other path is timed on the same inputs and reported under
 Under torchrun every rank decodes its own batch (weak scaling; sequences are
 independent, no data-path collective); the time is the max over ranks.
 
---impl reference times the fp64 CPU oracle (the reference arm of this build)
+--impl reference times the fp64 CPU oracle (the bench's reference arm)
 on the same workload: each step decodes one (sequence, group) unit of the
 batch, and its rate is scaled by the batch's number of such units.
 """

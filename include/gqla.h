@@ -59,7 +59,7 @@ extern "C" {
 typedef enum gqla_status {
   GQLA_OK = 0,
   GQLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, n_h % G != 0, s_q out of [1,4] */
-  GQLA_ERR_UNSUPPORTED = 2,  /* valid GQLA dims no kernel of this build handles */
+  GQLA_ERR_UNSUPPORTED = 2,  /* valid GQLA dims no kernel of this library handles */
   GQLA_ERR_ALIGNMENT = 3,    /* a pointer or row pitch below the 16-byte rule */
   GQLA_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than gqla_workspace_bytes */
   GQLA_ERR_CUDA = 5          /* a CUDA call or kernel launch failed */

@@ -295,7 +295,7 @@ const char* gqla_status_string(gqla_status s) {
   switch (s) {
     case GQLA_OK: return "GQLA_OK";
     case GQLA_ERR_INVALID_ARG: return "GQLA_ERR_INVALID_ARG: invalid argument";
-    case GQLA_ERR_UNSUPPORTED: return "GQLA_ERR_UNSUPPORTED: dims not handled by this build";
+    case GQLA_ERR_UNSUPPORTED: return "GQLA_ERR_UNSUPPORTED: dims not handled by this library";
     case GQLA_ERR_ALIGNMENT: return "GQLA_ERR_ALIGNMENT: pointer or pitch not 16-byte aligned";
     case GQLA_ERR_WORKSPACE: return "GQLA_ERR_WORKSPACE: workspace missing or too small";
     case GQLA_ERR_CUDA: return "GQLA_ERR_CUDA: CUDA launch failed";
