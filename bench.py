@@ -527,6 +527,12 @@ def run_ours(args):
     e2e_pipelined(3)
     torch.cuda.synchronize()
     e2e_ms = timed(lambda: e2e_pipelined(args.steps), 1) / args.steps
+    # both buffer sets hold what the plain step computes from the same inputs
+    step()
+    torch.cuda.synchronize()
+    for k in (0, 1):
+        if not (torch.equal(out_host2[k], out.cpu()) and torch.equal(lse_host2[k], lse.cpu())):
+            raise SystemExit("pipelined end-to-end step %d differs from the step's own result" % k)
     # the same, recorded once as a CUDA graph (copies included) and replayed
     e2e_graph_ms = None
     if not args.no_graph:
