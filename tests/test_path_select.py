@@ -15,22 +15,22 @@ B200 = (148, 6559.0, 1656.2)   # SMs, copy GB/s, dense bf16 TFLOP/s (measured on
 # d = v = 128, B32, L 32K), measured on one B200 with `bench.py --sweep
 # crossover` (absorb ms, GQA ms).  A performance record, not an oracle value.
 MEASURED_B200 = {
-    (1, 1): (0.493, 0.130), (1, 2): (0.938, 0.227), (1, 4): (1.738, 0.414),
-    (2, 1): (0.494, 0.236), (2, 2): (0.938, 0.235), (2, 4): (1.738, 0.416),
-    (4, 1): (0.493, 0.485), (4, 2): (0.938, 0.440), (4, 4): (1.739, 0.448),
-    (8, 1): (0.492, 0.747), (8, 2): (0.938, 0.852), (8, 4): (1.743, 0.861),
-    (16, 1): (0.502, 1.486), (16, 2): (0.938, 1.488), (16, 4): (1.738, 1.603),
-    (32, 1): (0.495, 2.938), (32, 2): (0.936, 2.950), (32, 4): (1.737, 2.978),
-    (128, 1): (0.501, 11.867), (128, 2): (0.939, 11.873), (128, 4): (1.738, 11.879),
+    (1, 1): (0.489, 0.133), (1, 2): (0.924, 0.227), (1, 4): (1.710, 0.413),
+    (2, 1): (0.488, 0.237), (2, 2): (0.922, 0.246), (2, 4): (1.710, 0.417),
+    (4, 1): (0.487, 0.485), (4, 2): (0.923, 0.460), (4, 4): (1.710, 0.476),
+    (8, 1): (0.487, 0.759), (8, 2): (0.923, 0.855), (8, 4): (1.712, 0.912),
+    (16, 1): (0.498, 1.509), (16, 2): (0.928, 1.512), (16, 4): (1.711, 1.615),
+    (32, 1): (0.502, 2.986), (32, 2): (0.930, 2.998), (32, 4): (1.723, 3.031),
+    (128, 1): (0.497, 12.161), (128, 2): (0.926, 12.171), (128, 4): (1.710, 12.175),
 }
 
 # The DeepSeek-V3-shaped layer (n_h 128, G 16, B64) over context lengths,
 # `bench.py --sweep context` on the same B200: (L, s_q) -> (absorb ms, GQA ms).
 MEASURED_CONTEXT_B200 = {
-    (8192, 1): (0.278, 0.770), (8192, 2): (0.532, 0.793),
-    (16384, 1): (0.504, 1.485), (16384, 2): (0.953, 1.509),
-    (32768, 1): (0.946, 2.928), (32768, 2): (1.743, 2.953),
-    (65536, 1): (1.740, 5.852), (65536, 2): (3.326, 5.877),
+    (8192, 1): (0.279, 0.779), (8192, 2): (0.531, 0.803),
+    (16384, 1): (0.501, 1.507), (16384, 2): (0.958, 1.532),
+    (32768, 1): (0.934, 2.978), (32768, 2): (1.744, 3.001),
+    (65536, 1): (1.728, 5.970), (65536, 2): (3.281, 6.001),
 }
 
 
@@ -76,8 +76,8 @@ def test_structure_of_the_estimates(G):
     # the shared-RoPE K pool streams fewer bytes
     assert _est(G, 128, 16, 1, 64, 16384, shared=True)[2] < _est(G, 128, 16, 1, 64, 16384)[2]
     # doubling the context nearly doubles both (long-context regime); the
-    # absorbed call's side GEMMs and merge do not grow with L (measured: 0.504
-    # -> 0.946 ms, a factor 1.88)
+    # absorbed call's side GEMMs and merge do not grow with L (measured: 0.501
+    # -> 0.934 ms, a factor 1.87)
     p1, a1, g1 = _est(G, 128, 16, 1, 64, 16384)
     p2, a2, g2 = _est(G, 128, 16, 1, 64, 32768)
     assert 1.7 < a2 / a1 < 2.1 and 1.9 < g2 / g1 < 2.1
