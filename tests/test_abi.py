@@ -99,6 +99,13 @@ def test_validation_before_launch(G):
     a = ctypes.c_void_p(0x10000)
     assert L.gqla_decode_gqa(ctypes.byref(d), ctypes.byref(lay), a, a, a, a, None, 4, a, 16, None,
                              None) == G.GQLA_ERR_WORKSPACE
+    # an empty batch, or a length bound below one token, is refused (B > 0 in the header)
+    for batch, max_len in ((0, 8192), (4, 0)):
+        empty = G.GqlaKvLayout(batch, lens.data_ptr(), max_len, 0, 8192, None, 0, 0)
+        assert L.gqla_decode_gqa(ctypes.byref(d), ctypes.byref(empty), a, a, a, a, None, 0, a, 1 << 30, None,
+                                 None) == G.GQLA_ERR_INVALID_ARG
+        assert L.gqla_decode_absorb(ctypes.byref(d), ctypes.byref(empty), a, a, a, a, a, None, 0, a, 1 << 30,
+                                    None, None) == G.GQLA_ERR_INVALID_ARG
     # paged layout without a block table
     bad = G.GqlaKvLayout(4, lens.data_ptr(), 8192, 64, 0, None, 0, 0)
     assert L.gqla_decode_gqa(ctypes.byref(d), ctypes.byref(bad), a, a, a, a, None, 0, a, 1 << 30, None,
