@@ -84,6 +84,29 @@ def test_bf16_absorb_merge_row_tiles(B):
     H.check_units(inp, out, lse, H.sample_units(inp, 6, seed=B), "absorb merge tiles B=%d" % B)
 
 
+@pytest.mark.parametrize("page", [128, 256])
+@pytest.mark.parametrize("path", ["absorb", "gqa"])
+def test_bf16_large_pages(page, path):
+    """Pages of 128 and 256 tokens (any multiple of the 64-token tile):
+    lengths that end inside a page, on a page boundary and past several
+    pages, through a permuted block table."""
+    d = synth.Dims(**DSV3, s_q=2)
+    inp = _wl(d, 3, [130, 2 * page, 1500], page=page, seed=page)
+    out, lse = H.run_decode(inp, path)
+    H.check_units(inp, out, lse, H.sample_units(inp, 6, seed=page), "dsv3 bf16 %s page=%d" % (path, page))
+
+
+@pytest.mark.parametrize("G", [1, 2])
+@pytest.mark.parametrize("splits", [0, 3])
+def test_gqa_wide_three_new_tokens(G, splits):
+    """The tcgen05 GQA kernel at s_q 3: 384 rows a group at G 1 (three full
+    128-row blocks), 192 at G 2 (the second block half empty), paged."""
+    d = synth.Dims(n_h=128, G=G, d_nope=128, d_rope=64, d_v=128, r=512, s_q=3)
+    inp = _wl(d, 2, [300, 777], page=128, seed=50 + G)
+    out, lse = H.run_decode(inp, "gqa", num_splits=splits)
+    H.check_units(inp, out, lse, H.sample_units(inp, 4, seed=G), "gqa_wide G=%d s_q=3 splits=%d" % (G, splits))
+
+
 @pytest.mark.parametrize("G", [1, 2, 4, 32, 128])
 @pytest.mark.parametrize("s_q", [1, 4])
 def test_bf16_group_counts(G, s_q):
