@@ -72,4 +72,33 @@ void count_launch(int n = 1);
 // Raises a kernel's dynamic shared-memory limit once per device.
 cudaError_t ensure_smem_limit(const void* func, int bytes);
 
+namespace ptx {
+// A kernel launched by launch_pdl may begin while the kernel ahead of it on the
+// stream is still running.  pdl_wait() returns once that kernel has completed
+// and its memory writes are visible (at once when the launch had no such
+// dependency); pdl_trigger() lets the next such kernel begin launching once
+// every CTA of this grid has called it or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+}  // namespace ptx
+
+// Launches a kernel that may begin before the kernel ahead of it on the stream
+// has finished (programmatic stream serialisation): the kernel reads that
+// kernel's results only after ptx::pdl_wait().
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 }  // namespace gqla

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x;
   const int b = blockIdx.y / p.hblocks, hb = blockIdx.y % p.hblocks;
+  ptx::pdl_trigger();   // the merge may launch once every CTA of this grid has started
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&q_full, 4);
@@ -229,7 +230,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Q~ = [q~ (512) ; q_rope (64)] of each row into TMEM (lanes 0-15, one
     // row per lane), as bf16 pairs; lanes 16-31 store zeros into the O
-    // half-lanes, which the first PV overwrites.
+    // half-lanes, which the first PV overwrites.  q~ comes from the launch
+    // ahead of this one, which may still be running (the latent loads above
+    // do not depend on it).
+    ptx::pdl_wait();
     {
       const int row_q = 16 * qd + (lane & 15);
       const bool load = lane < 16 && hb * kM + row_q < p.rows_unit && grow0 + row_q < p.rows;
@@ -454,9 +458,9 @@ cudaError_t tc_absorb_decode(const Problem& p, const void* q, const void* latent
   e = ensure_smem_limit((const void*)absorb_decode_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(S, p.ly.batch * prm.hblocks);
-  absorb_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(kv_map, prm);
+  e = launch_pdl(absorb_decode_kernel, grid, dim3(kThreads), kSmemBytes, s, kv_map, prm);
   count_launch();
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (gemm_combine_up_supports(p))
     return combine_up_mma(p, S, w.o_part, w.lse_part, W_uv, out, lse, s);

@@ -57,6 +57,7 @@ constexpr int kAqRows = 64, kAqN = 128, kAqMaxK = 256, kAqThreads = 256;
 __global__ void __launch_bounds__(kAqThreads) absorb_q_mma_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_uk,
                                                            bf16* __restrict__ qt, int rows_g, int n_h, int m,
                                                            int d_n, int d_qk, int r) {
+  ptx::pdl_trigger();   // the decode may launch and start its loads meanwhile
   extern __shared__ __align__(16) uint8_t sm[];
   const int g = blockIdx.z, n0 = blockIdx.y * kAqN;
   const int pitch = (d_n + 8) * 2;
@@ -143,6 +144,8 @@ __global__ void __launch_bounds__(kUpThreads) merge_up_kernel(int S, const float
     cp_async16(b + kk * kUpBpitch + c * 16, Wg + (size_t)kk * kUpN + c * 8, true);
   }
   cp_async_commit();
+  // the decode's partials are read from here on (W_uv^g is already on its way)
+  ptx::pdl_wait();
 
   // merge: a warp per row, a lane on 4 columns of each 128-column quarter
   for (int rr = warp; rr < kUpRows; rr += kUpThreads / 32) {
@@ -270,13 +273,16 @@ cudaError_t combine_up_mma(const Problem& p, int S, const float* o_part, const f
   const bf16* w = (const bf16*)W_uv;
   bf16* o = (bf16*)out;
   if (R == 64)
-    merge_up_kernel<64><<<grid, kUpThreads, up_smem(64), s>>>(S, o_part, lse_part, w, o, lse_out, p.rows, rows_g, d.n_h, p.m);
+    e = launch_pdl(merge_up_kernel<64>, grid, dim3(kUpThreads), up_smem(64), s, S, o_part, lse_part, w, o, lse_out, p.rows,
+                   rows_g, d.n_h, p.m);
   else if (R == 32)
-    merge_up_kernel<32><<<grid, kUpThreads, up_smem(32), s>>>(S, o_part, lse_part, w, o, lse_out, p.rows, rows_g, d.n_h, p.m);
+    e = launch_pdl(merge_up_kernel<32>, grid, dim3(kUpThreads), up_smem(32), s, S, o_part, lse_part, w, o, lse_out, p.rows,
+                   rows_g, d.n_h, p.m);
   else
-    merge_up_kernel<16><<<grid, kUpThreads, up_smem(16), s>>>(S, o_part, lse_part, w, o, lse_out, p.rows, rows_g, d.n_h, p.m);
+    e = launch_pdl(merge_up_kernel<16>, grid, dim3(kUpThreads), up_smem(16), s, S, o_part, lse_part, w, o, lse_out, p.rows,
+                   rows_g, d.n_h, p.m);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace gqla
