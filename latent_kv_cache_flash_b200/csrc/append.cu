@@ -14,6 +14,10 @@ namespace {
 template <typename T>
 __global__ void append_rows_kernel(KvLayout ly, const T* __restrict__ new_rows, T* __restrict__ latent, int s_q,
                                    int E, int32_t* st) {
+  // launched while the kernel ahead of it may still run: wait for it before
+  // any memory access, then let the next kernel launch
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const int b = blockIdx.x / s_q, i = blockIdx.x % s_q;
   const int L = seq_len_checked(ly, b, s_q, i == 0 ? st : nullptr);
   if (L < 0) return;
@@ -34,13 +38,15 @@ __global__ void append_rows_kernel(KvLayout ly, const T* __restrict__ new_rows, 
 
 cudaError_t append_rows(const Problem& p, const void* new_rows, void* latent, int32_t* st, cudaStream_t s) {
   const int blocks = p.ly.batch * p.d.s_q;
+  cudaError_t e;
   if (p.d.dtype == GQLA_F32)
-    append_rows_kernel<float><<<blocks, 64, 0, s>>>(p.ly, (const float*)new_rows, (float*)latent, p.d.s_q, p.E, st);
+    e = launch_pdl(append_rows_kernel<float>, dim3(blocks), dim3(64), 0, s, p.ly, (const float*)new_rows,
+                   (float*)latent, p.d.s_q, p.E, st);
   else
-    append_rows_kernel<__nv_bfloat16><<<blocks, 64, 0, s>>>(p.ly, (const __nv_bfloat16*)new_rows,
-                                                            (__nv_bfloat16*)latent, p.d.s_q, p.E, st);
+    e = launch_pdl(append_rows_kernel<__nv_bfloat16>, dim3(blocks), dim3(64), 0, s, p.ly,
+                   (const __nv_bfloat16*)new_rows, (__nv_bfloat16*)latent, p.d.s_q, p.E, st);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace gqla

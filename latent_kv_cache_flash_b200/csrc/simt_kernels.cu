@@ -201,6 +201,10 @@ __global__ void up_proj_kernel(const float* __restrict__ o_lat, const T* __restr
 template <typename T>
 __global__ void combine_kernel(int S, long long rows, int D, const float* __restrict__ o_part,
                                const float* __restrict__ lse_part, T* __restrict__ out, float* __restrict__ lse_out) {
+  // launched while the kernel ahead of it may still run: wait for it before
+  // any memory access, then let the next kernel launch
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -306,13 +310,15 @@ cudaError_t combine(int S, long long rows, int D, const float* o_part, const flo
                     gqla_dtype out_dtype, float* lse_out, cudaStream_t s) {
   const int wpb = 8;
   unsigned blocks = (unsigned)((rows + wpb - 1) / wpb);
+  cudaError_t e;
   if (out_dtype == GQLA_F32)
-    combine_kernel<float><<<blocks, 32 * wpb, 0, s>>>(S, rows, D, o_part, lse_part, (float*)out, lse_out);
+    e = launch_pdl(combine_kernel<float>, dim3(blocks), dim3(32 * wpb), 0, s, S, rows, D, o_part, lse_part,
+                   (float*)out, lse_out);
   else
-    combine_kernel<__nv_bfloat16><<<blocks, 32 * wpb, 0, s>>>(S, rows, D, o_part, lse_part,
-                                                              (__nv_bfloat16*)out, lse_out);
+    e = launch_pdl(combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(32 * wpb), 0, s, S, rows, D, o_part, lse_part,
+                   (__nv_bfloat16*)out, lse_out);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace gqla

@@ -145,6 +145,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     expand_tc_kernel(const __grid_constant__ CUtensorMap lat_map, const __grid_constant__ CUtensorMap uk_map,
                      const __grid_constant__ CUtensorMap uv_map, const __grid_constant__ CUtensorMap k_store,
                      const __grid_constant__ CUtensorMap v_store, const ExpandParams p) {
+  // launched while the kernel ahead of it may still run: wait for it before
+  // any memory access, then let the next kernel launch
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], acc_full[2], acc_empty[2], drain;
@@ -823,9 +827,10 @@ cudaError_t tc_expand(const Problem& p, const void* latent, const void* W_uk, co
   if (e != cudaSuccess) return e;
   const long long grid = prm.n_items < num_sms() ? prm.n_items : num_sms();
   if (grid < 1) return cudaSuccess;
-  expand_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(lat_map, uk_map, uv_map, k_store, v_store, prm);
+  e = launch_pdl(expand_tc_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, lat_map, uk_map, uv_map,
+                 k_store, v_store, prm);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t tc_expand_dense(const Problem& p, const void* rows, void* k_pool, void* v_pool, const void* W_uk,
@@ -858,9 +863,10 @@ cudaError_t tc_expand_dense(const Problem& p, const void* rows, void* k_pool, vo
   cudaError_t e = ensure_smem_limit((const void*)expand_tc_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long grid = prm.n_items < num_sms() ? prm.n_items : num_sms();
-  expand_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(lat_map, uk_map, uv_map, k_store, v_store, prm);
+  e = launch_pdl(expand_tc_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, lat_map, uk_map, uv_map,
+                 k_store, v_store, prm);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace gqla

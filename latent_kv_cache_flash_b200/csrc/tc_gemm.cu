@@ -57,7 +57,10 @@ constexpr int kAqRows = 64, kAqN = 128, kAqMaxK = 256, kAqThreads = 256;
 __global__ void __launch_bounds__(kAqThreads) absorb_q_mma_kernel(const bf16* __restrict__ q, const bf16* __restrict__ W_uk,
                                                            bf16* __restrict__ qt, int rows_g, int n_h, int m,
                                                            int d_n, int d_qk, int r) {
-  ptx::pdl_trigger();   // the decode may launch and start its loads meanwhile
+  // launched while the kernel ahead of it may still run: wait for it before
+  // any memory access, then let the decode launch and start its loads
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   extern __shared__ __align__(16) uint8_t sm[];
   const int g = blockIdx.z, n0 = blockIdx.y * kAqN;
   const int pitch = (d_n + 8) * 2;
@@ -131,6 +134,7 @@ __global__ void __launch_bounds__(kUpThreads) merge_up_kernel(int S, const float
                                                               float* __restrict__ lse_out, long long rows,
                                                               int rows_g, int n_h, int m) {
   extern __shared__ __align__(16) uint8_t sm[];
+  ptx::pdl_trigger();   // the next call's first kernel may launch (it waits for this one)
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t a = ptx::smem_u32(sm), b = a + kUpRows * kUpApitch;
@@ -245,10 +249,10 @@ cudaError_t absorb_q_mma(const Problem& p, const void* q, const void* W_uk, bf16
   cudaError_t e = ensure_smem_limit((const void*)absorb_q_mma_kernel, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((rows_g + kAqRows - 1) / kAqRows, d.r / kAqN, d.G);
-  absorb_q_mma_kernel<<<grid, kAqThreads, smem, s>>>((const bf16*)q, (const bf16*)W_uk, qt, rows_g, d.n_h, p.m, d.d_nope,
-                                              p.d_qk, d.r);
+  e = launch_pdl(absorb_q_mma_kernel, grid, dim3(kAqThreads), smem, s, (const bf16*)q, (const bf16*)W_uk, qt, rows_g,
+                 d.n_h, p.m, d.d_nope, p.d_qk, d.r);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 bool gemm_combine_up_supports(const Problem& p) {

@@ -71,6 +71,10 @@ static_assert(kConsumerWarps * 16 * kOStride * 4 + 2 * kConsumerWarps * 16 * 4 <
 __global__ void __launch_bounds__(kThreads, 2)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                       const GqaParams p) {
+  // launched while the kernel ahead of it may still run: wait for it before
+  // any memory access, then let the next kernel launch
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) uint64_t full_bar[kStages];
@@ -446,8 +450,9 @@ cudaError_t tc_gqa_decode(const Problem& p, const void* q, const void* k_pool, c
   }
   cudaError_t e = ensure_smem_limit((const void*)gqa_decode_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  gqa_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, prm);
+  e = launch_pdl(gqa_decode_kernel, grid, dim3(kThreads), kSmemBytes, s, kmap, vmap, prm);
   count_launch();
+  if (e != cudaSuccess) return e;
   if (merge && merged) *merged = true;
   return cudaGetLastError();
 }

@@ -75,6 +75,10 @@ struct WideParams {
 __global__ void __launch_bounds__(kThreads, 1)
     gqa_wide_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                     const WideParams p) {
+  // launched while the kernel ahead of it may still run: wait for it before
+  // any memory access, then let the next kernel launch
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sK = smem;
@@ -494,8 +498,9 @@ cudaError_t tc_gqa_wide_decode(const Problem& p, const void* q, const void* k_po
   cudaError_t e = ensure_smem_limit((const void*)gqa_wide_kernel, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.plan.num_splits * prm.rblocks, p.ly.batch * d.G);
-  gqa_wide_kernel<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, prm);
+  e = launch_pdl(gqa_wide_kernel, grid, dim3(kThreads), kSmemBytes, s, kmap, vmap, prm);
   count_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
