@@ -23,7 +23,13 @@
  *    library-owned __device__ array (described at that call).  Host structs
  *    are read during the call only.
  *  - Work is queued on `stream` (a cudaStream_t; NULL = legacy default stream)
- *    and runs asynchronously; no call synchronises.
+ *    and runs asynchronously; no call synchronises.  The tensor-core kernels
+ *    are launched with programmatic stream serialisation: each call's first
+ *    kernel waits for all earlier work on the stream before touching memory,
+ *    and later kernels of the call may begin while their predecessor ends.
+ *    Work the caller queues afterwards sees the call's results in stream
+ *    order, except a kernel the caller itself launches with that attribute,
+ *    which (as any such kernel) must execute griddepcontrol.wait first.
  *  - Arguments are validated on the host before any launch; a failed check
  *    returns a status and launches nothing.  A kernel launch failure returns
  *    GQLA_ERR_CUDA.
