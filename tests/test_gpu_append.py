@@ -164,3 +164,41 @@ def test_append_flags_bad_sequences_and_skips_them():
     assert flags & gqla.DEV_SHORT_SEQ and flags & gqla.DEV_BAD_PAGE
     # sequence 1 rewrote its own (identical) rows, 0 and 2 wrote nothing
     assert torch.equal(inp.latent, before)
+
+
+@pytest.mark.parametrize("shape", ["llama", "wide"])
+@pytest.mark.parametrize("page", [0, 64])
+def test_chained_calls_without_host_sync(shape, page):
+    # the append, then both decode paths, queued back to back on one stream
+    # with no host synchronisation: every call must see all that the one
+    # before it wrote (its kernels may launch early, but the first waits for
+    # the kernel ahead before any access).  New slots are poisoned first, so a
+    # decode that read too early would differ from the synchronised run.
+    dims_kw = LLAMA if shape == "llama" else dict(n_h=128, G=2, d_nope=128, d_rope=64, d_v=128, r=512)
+    d = synth.Dims(**dims_kw, s_q=2)
+    inp = _inputs(d, [700, 66, 1029, 2048], page, seed=77)
+    kp0, vp0 = H.run_expand(inp)
+    new_rows = _new_rows(inp)
+    lat0 = inp.latent.clone()
+
+    def run(sync):
+        inp.latent.copy_(lat0)
+        kp, vp = kp0.clone(), vp0.clone()
+        for t in (inp.latent, kp, vp):
+            _poison_new_slots(t, inp)
+        if sync:
+            torch.cuda.synchronize()
+        _append(inp, new_rows, inp.latent, (kp, vp))
+        if sync:
+            torch.cuda.synchronize()
+        res = [H.run_decode(inp, "absorb")]
+        if sync:
+            torch.cuda.synchronize()
+        res.append(H.run_decode(inp, "gqa", pools=(kp, vp)))
+        torch.cuda.synchronize()
+        return res
+
+    ref = run(True)
+    for _ in range(3):
+        for (o1, l1), (o2, l2) in zip(ref, run(False)):
+            assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
