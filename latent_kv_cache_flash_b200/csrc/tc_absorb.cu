@@ -135,15 +135,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n_tiles > 0) {
       ptx::prefetch_tmap(&kv_map);
       int issued = 0;
+      // a tile's pool row (a page-table read when paged) is looked up one
+      // tile ahead, so its latency overlaps the wait for the slot
+      int row_next = (int)token_row(p.ly, b, t_begin, nullptr);
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kStages, k = j / kStages;
+        const int row0 = row_next;
+        if (j + 1 < n_tiles) row_next = (int)token_row(p.ly, b, t_begin + (j + 1) * kTk, nullptr);
         if (k > 0 && !ptx::mbar_wait(&kv_empty[s], (k - 1) & 1)) {
           flag_status(p.st, GQLA_DEV_TIMEOUT);
           atomicExch(&abort_flag, 1);
           break;
         }
         if (*(volatile int*)&abort_flag) break;
-        const int row0 = (int)token_row(p.ly, b, t_begin + j * kTk, nullptr);
         uint8_t* dst = sKV + s * kStageBytes;
         ptx::mbar_arrive_expect_tx(&kv_full[s], (c_hi - c_lo) * kKVChunk);
         for (int c = c_lo; c < c_hi; ++c) ptx::tma_load_2d(dst + c * kKVChunk, &kv_map, &kv_full[s], 64 * c, row0);

@@ -106,16 +106,19 @@ __global__ void __launch_bounds__(kThreads, 2)
       ptx::prefetch_tmap(&kmap);
       ptx::prefetch_tmap(&vmap);
       const int kx = p.kr.nope_at(g), kxr = p.kr.rope_at(g), vx = g * kDv;
+      // a tile's pool row (a page-table read when paged) is looked up one
+      // tile ahead, so its latency overlaps the wait for the slot
+      int row_next = n_tiles > 0 ? (int)token_row(p.ly, b, t_begin, nullptr) : 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kStages, k = j / kStages;
+        const int row0 = row_next;
+        if (j + 1 < n_tiles) row_next = (int)token_row(p.ly, b, t_begin + (j + 1) * kT, nullptr);
         if (k > 0 && !ptx::mbar_wait(&empty_bar[s], (k - 1) & 1)) {
           flag_status(p.st, GQLA_DEV_TIMEOUT);
           atomicExch(&abort_flag, 1);
           break;
         }
         if (*(volatile int*)&abort_flag) break;
-        const int t0 = t_begin + j * kT;
-        const int row0 = (int)token_row(p.ly, b, t0, nullptr);
         uint8_t* st = smem + s * kStageBytes;
         ptx::mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
         // K: the group's two d_nope chunks, then its RoPE chunk; V: two chunks

@@ -143,15 +143,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n_tiles > 0) {
       ptx::prefetch_tmap(kside ? &kmap : &vmap);
       int issued = 0;
+      // a tile's pool row (a page-table read when paged) is looked up one
+      // tile ahead, so its latency overlaps the wait for the slot
+      int row_next = (int)token_row(p.ly, b, t_begin, nullptr);
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % nst, k = j / nst;
+        const int row0 = row_next;
+        if (j + 1 < n_tiles) row_next = (int)token_row(p.ly, b, t_begin + (j + 1) * kT, nullptr);
         if (k > 0 && !ptx::mbar_wait(&empty[s], (k - 1) & 1)) {
           flag_status(p.st, GQLA_DEV_TIMEOUT);
           atomicExch(&abort_flag, 1);
           break;
         }
         if (*(volatile int*)&abort_flag) break;
-        const int row0 = (int)token_row(p.ly, b, t_begin + j * kT, nullptr);
         if (kside) {
           uint8_t* dst = sK + s * kKSlotBytes;
           ptx::mbar_arrive_expect_tx(&full[s], kKSlotBytes);
